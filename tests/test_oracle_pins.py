@@ -267,7 +267,9 @@ def _all_bf16_patterns_no_nan():
     return b
 
 
-@pytest.mark.parametrize("scale", [0.05, 1.0, 0.37, 3.0])
+# 7.0 and 0.9 are scales for which x * (1/scale) and x / scale give different
+# e4m3 bytes for some bf16 x (60 and 30 of them), so a reciprocal-multiply fails here.
+@pytest.mark.parametrize("scale", [0.05, 1.0, 0.37, 3.0, 7.0, 0.9])
 def test_e4m3_exhaustive_bf16_through_entry_point(scale):
     """All bf16 patterns in q_nope (8 x 16 x 512 = 65536), flags Q_FP8|KV_FP8:
     each output byte equals torch's e4m3 cast of the fp32 quotient x / scale,
