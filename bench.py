@@ -1,0 +1,629 @@
+"""Benchmark of the fused MLA decode epilogue on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-sweep] [--no-cpu-baseline]
+
+One step is one call of the epilogue (the whole hot path) on one batch of
+the workload.  Default workload: the row-split boundary case, T=64 tokens,
+H=16 heads, bf16, RoPE (the decode size at which the vLLM PR #54896 report
+switches to three warps per row).  Inputs are device-resident when the timed
+region starts; consecutive steps rotate over input sets whose total is more
+than twice the L2, so every step reads HBM.  The K calls are replayed from
+CUDA graphs on one stream and timed with CUDA events on that stream; the
+bare-launch floor is an empty kernel with the same grid, block and launch
+attributes, timed the same way.
+
+Printed: one JSON line (rank 0) with the metric in microseconds per call,
+achieved HBM GB/s against the measured copy bandwidth, the launch floor, a
+sweep over the other workload sizes, the end-to-end time through the Python
+API with pinned host buffers, the CPU oracle as a baseline and the SM clocks
+seen under load.  ``--impl reference`` times the CPU oracle instead (the only
+reference implementation this operation has here).
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime as _dt
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mla_decode_attention_10_b200 import workloads as W  # noqa: E402
+
+METRIC = "µs/call and achieved HBM GB/s (fraction of ~8 TB/s) vs T for MLA epilogue"
+UNIT = "µs/call"
+HEADLINE = "split_boundary_t64_h16_rope"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+GRAPH_CALLS = 500
+
+
+# ---------------------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------------------
+
+def rank_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def job_us_per_call(max_ms: float, steps: int, world: int) -> float:
+    """Whole-job microseconds per call: every rank makes `steps` calls in at
+    most `max_ms`, so the job completes world*steps calls in that time."""
+    return max_ms * 1e3 / (steps * world)
+
+
+# ---------------------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms in the background (read-only queries)."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        try:
+            self.gpu = f"GPU-{torch.cuda.get_device_properties(gpu_index).uuid}"
+        except Exception:
+            self.gpu = str(gpu_index)
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def samples(self):
+        out = []
+        if not self.path or not os.path.exists(self.path):
+            return out
+        for row in csv.reader(open(self.path)):
+            if len(row) < 10:
+                continue
+            try:
+                ts = _dt.datetime.strptime(row[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                out.append(dict(t=ts, sm=float(row[2]), sm_max=float(row[3]), power=float(row[4]),
+                                hw=row[6].strip(), hw_thermal=row[7].strip(), sw_thermal=row[8].strip(),
+                                sw_power=row[9].strip()))
+            except ValueError:
+                continue
+        return out
+
+    def summary(self, t0: float, t1: float):
+        s = self.samples()
+        inside = [x for x in s if t0 <= x["t"] <= t1]
+        window = "timed region"
+        if not inside:
+            inside = [x for x in s if x["power"] > 0 and t0 - 3.0 <= x["t"] <= t1 + 1.0]
+            window = "load of the same graphs within 3 s before the timed region (region too short to sample)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": "no samples"}
+        reasons = set()
+        for x in inside:
+            for k, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                            ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if x[k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x["sm"] for x in inside),
+                "sm_max_mhz": max(x["sm_max"] for x in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
+
+
+# ---------------------------------------------------------------------------------------
+# device timing
+# ---------------------------------------------------------------------------------------
+
+def capture(step_fn, first: int, n: int, stream) -> torch.cuda.CUDAGraph:
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step_fn(first + i)
+    return g
+
+
+def graph_plan(steps: int):
+    """Graphs of at most GRAPH_CALLS calls covering `steps` calls."""
+    full, rest = divmod(steps, GRAPH_CALLS)
+    return [GRAPH_CALLS] * full + ([rest] if rest else [])
+
+
+class GraphRunner:
+    def __init__(self, step_fn, steps: int, stream):
+        self.stream = stream
+        self.graphs = []
+        first = 0
+        for n in graph_plan(steps):
+            self.graphs.append(capture(step_fn, first, n, stream))
+            first += n
+
+    def replay(self):
+        for g in self.graphs:
+            g.replay()
+
+
+def timed(runner: GraphRunner, device) -> float:
+    """ms for one replay of all graphs, bracketed by barrier + synchronize, max over ranks."""
+    s = runner.stream
+    flush_l2()
+    barrier(device)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        runner.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    barrier(device)
+    return max_over_ranks(e0.elapsed_time(e1), device)
+
+
+def measured_hbm_gbs():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = float(json.load(open(p))["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs: torch copy, read+write bytes)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+# ---------------------------------------------------------------------------------------
+# workloads on the device
+# ---------------------------------------------------------------------------------------
+
+def named_variant(name: str, seed_offset: int) -> W.Workload:
+    """The named workload's recipe with its seed shifted (fresh values, same shapes)."""
+    return W.named(name, seed_offset)
+
+
+class DeviceSets:
+    """Input sets of one workload on the device, each a complete set of call
+    arguments, so that consecutive calls read different memory.
+
+    Sizes whose one call already touches more than 2x L2 get two full copies
+    of the named workload.  Smaller ones get S sets cut from device pools
+    drawn with a seeded CUDA generator (same shapes and distributions as the
+    named recipe, contiguous layouts), S chosen so that S calls touch more
+    than 2x L2; the RoPE table and the cache are shared by all sets (each
+    call writes its own T slots)."""
+
+    def __init__(self, name: str):
+        self.name = name
+        self.w0 = w0 = named_variant(name, 0)
+        self.bytes_per_call = w0.algorithmic_bytes()
+        self.sets = []
+        if self.bytes_per_call > 2 * L2_BYTES or w0.producer or not w0.q_nope.is_contiguous():
+            table = w0.cos_sin.to("cuda") if w0.cos_sin is not None else None
+            for k in range(2):
+                w = w0 if k == 0 else named_variant(name, k)
+                w.cos_sin = None
+                d = w.to("cuda")
+                d.cos_sin = table
+                q_out = torch.empty((w.T, w.H, W.ROW), dtype=w.q_out_dtype(), device="cuda")
+                src = (d.q_nope.contiguous().clone(), d.q_pe.contiguous().clone()) if w.producer else None
+                self.sets.append((d, q_out, src))
+            self.touched = 2 * self.bytes_per_call
+            return
+        S = max(2, -(-2 * L2_BYTES // self.bytes_per_call))
+        self._pool(w0, S)
+
+    def _pool(self, w0, S):
+        T, H = w0.T, w0.H
+        g = torch.Generator(device="cuda").manual_seed(1234 + T)
+        std = float(w0.q_nope.float().std()) if w0.q_nope.numel() > 1 else 1.0
+        std = 2.0 if std > 1.5 else 1.0
+
+        def randn(*shape):
+            return (torch.randn(*shape, generator=g, device="cuda") * std).to(torch.bfloat16)
+
+        qn, qp, kv, kp = randn(S, T, H, W.NOPE), randn(S, T, H, W.PE), randn(S, T, W.NOPE), randn(S, T, W.PE)
+        cap = w0.num_blocks * w0.block_size
+        if S * T <= cap:
+            slots = torch.randperm(cap, generator=g, device="cuda")[:S * T].view(S, T)
+        else:
+            slots = torch.argsort(torch.rand(S, cap, generator=g, device="cuda"), dim=1)[:, :T]
+        slots = slots.to(torch.int64).contiguous()
+        pos = None
+        table = None
+        if w0.flags & W.FLAG_ROPE:
+            rows = w0.cos_sin.shape[0]
+            pos = torch.randint(0, rows, (S, T), generator=g, device="cuda", dtype=torch.int32)
+            table = w0.cos_sin.to("cuda")
+        cache = w0.cache.to("cuda")
+        qs = w0.q_scale.to("cuda") if w0.q_scale is not None else None
+        ks = w0.kv_scale.to("cuda") if w0.kv_scale is not None else None
+        q_out = torch.empty((S, T, H, W.ROW), dtype=w0.q_out_dtype(), device="cuda")
+        self._keep = (qn, qp, kv, kp, slots, pos, q_out)
+        for k in range(S):
+            d = W.Workload(name=w0.name, T=T, H=H, block_size=w0.block_size, num_blocks=w0.num_blocks,
+                           flags=w0.flags, q_nope=qn[k], q_pe=qp[k], kv_c=kv[k], k_pe=kp[k],
+                           slot_mapping=slots[k], cache=cache, positions=None if pos is None else pos[k],
+                           cos_sin=table, q_scale=qs, kv_scale=ks)
+            self.sets.append((d, q_out[k], None))
+        self.touched = S * self.bytes_per_call
+
+
+def flush_l2():
+    """Write a buffer of twice the L2 size (outside any timed region)."""
+    buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device="cuda")
+    buf.fill_(1)
+    torch.cuda.synchronize()
+    del buf
+
+
+# ---------------------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    from mla_decode_attention_10_b200 import epilogue as E
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    E.lib()  # fail loudly if the CUDA library is missing
+    stream = torch.cuda.Stream(device)
+    peak, peak_note = measured_hbm_gbs()
+
+    def epilogue_step(ds, extra=0):
+        def f(i):
+            d, q_out, _ = ds.sets[i % len(ds.sets)]
+            rc = E.launch_workload(d, q_out, extra_flags=extra, stream=stream)
+            if rc != E.MLA_OK:
+                raise E.MlaError(rc, "mla_epilogue_launch")
+        return f
+
+    def floor_step(T, H, flags):
+        plan = E.mla_epilogue_plan(T, H, flags)
+
+        def f(i):
+            rc = E.mla_harness_empty(plan.blocks, plan.threads_per_block, flags & E.MLA_FLAG_PDL, stream.cuda_stream)
+            if rc != E.MLA_OK:
+                raise E.MlaError(rc, "mla_harness_empty")
+        return f, plan
+
+    def measure(step, steps, warmup):
+        warm = GraphRunner(step, max(warmup, 1), stream)
+        warm.replay()
+        torch.cuda.synchronize()
+        runner = GraphRunner(step, steps, stream)
+        runner.replay()  # first replay uploads the graphs
+        torch.cuda.synchronize()
+        return runner
+
+    # ---- headline workload
+    ds = DeviceSets(args.workload)
+    w0 = ds.w0
+    step = epilogue_step(ds)
+    runner = measure(step, args.steps, args.warmup)
+    fstep, plan = floor_step(w0.T, w0.H, 0)
+    frunner = measure(fstep, args.steps, args.warmup)
+    for _ in range(args.warmup):
+        runner.replay()
+    torch.cuda.synchronize()
+
+    with ClockSampler(local_rank) as clk:
+        # a short soak of the same graphs so that clocks are sampled under this load
+        t_soak = time.time()
+        while time.time() - t_soak < 1.5:
+            runner.replay()
+            torch.cuda.synchronize()
+        t0 = time.time()
+        ms = timed(runner, device)
+        t1 = time.time()
+        time.sleep(0.25)
+    clocks = clk.summary(t0, t1)
+    floor_ms = timed(frunner, device)
+
+    us = job_us_per_call(ms, args.steps, world)
+    per_call_us_rank = ms * 1e3 / args.steps
+    gbs = w0.algorithmic_bytes() / (per_call_us_rank * 1e-6) / 1e9
+    floor_us = floor_ms * 1e3 / args.steps
+
+    # PDL-chained variant of the same call sequence (each call a programmatic
+    # dependent of the previous one; sets are disjoint, so the contract holds)
+    prunner = measure(epilogue_step(ds, E.MLA_FLAG_PDL), args.steps, args.warmup)
+    pfstep, _ = floor_step(w0.T, w0.H, E.MLA_FLAG_PDL)
+    pfrunner = measure(pfstep, args.steps, args.warmup)
+    pdl_us = timed(prunner, device) * 1e3 / args.steps
+    pdl_floor_us = timed(pfrunner, device) * 1e3 / args.steps
+    del prunner, pfrunner
+
+    # ---- end to end through the Python API: pinned host inputs -> call -> q_out to host
+    e2e = run_e2e(args, w0, stream, device, world)
+
+    # ---- sweep of the other sizes (their own bench lines are not printed; this is context)
+    sweep = []
+    if not args.no_sweep:
+        for name in sweep_names(args.workload):
+            sweep.append(sweep_one(name, E, stream, device, peak, epilogue_step, floor_step, measure))
+            torch.cuda.empty_cache()
+
+    line = {
+        "metric": METRIC, "value": round(us, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "T": w0.T, "H": w0.H, "flags": flag_names(w0.flags),
+                   "recipe": w0.recipe, "mode": "split" if plan.mode == E.MLA_MODE_SPLIT else "rows",
+                   "grid": [plan.blocks, plan.threads_per_block],
+                   "l2": f"inputs larger than L2: {len(ds.sets)} rotating input sets touching "
+                         f"{ds.touched / 2 ** 20:.0f} MiB (> 2x L2); L2 written over before each timed region",
+                   "timing": f"CUDA graphs of <= {GRAPH_CALLS} calls on one stream, CUDA events",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "gbs": round(gbs, 1),
+        "launch_floor_us": round(floor_us, 4),
+        "floor_ratio": round(per_call_us_rank / floor_us, 3),
+        "pdl_chain": {"us_per_call": round(pdl_us, 4), "floor_us": round(pdl_floor_us, 4),
+                      "floor_ratio": round(pdl_us / pdl_floor_us, 3)},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None,
+                     "peak_source": peak_note,
+                     "note": "decode-size call: launch and memory latency bound, not bandwidth bound; "
+                             "see sweep for the bandwidth-bound sizes"},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "sweep": sweep,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(args.workload)
+    return line
+
+
+def flag_names(f: int) -> str:
+    names = [n for bit, n in ((W.FLAG_ROPE, "rope"), (W.FLAG_Q_FP8, "q_fp8"), (W.FLAG_KV_FP8, "kv_fp8"))
+             if f & bit]
+    return "+".join(names) if names else "none"
+
+
+def sweep_names(headline: str):
+    names = ["decode_t4_h16", "split_boundary_t64_h16_rope", "split_boundary_t65_h16_rope"]
+    names += [f"decode_sweep_t{t}_h16_rope_fp8" for t in W.DECODE_SWEEP_T]
+    names += ["prefill_t1024_h128_strided", "batch_t8192_h16_pdl_fp8"]
+    return [n for n in names if n != headline]
+
+
+def sweep_one(name, E, stream, device, peak, epilogue_step, floor_step, measure, steps=None):
+    ds = DeviceSets(name)
+    w0 = ds.w0
+    big = w0.algorithmic_bytes() > 32 * 2 ** 20
+    n = steps or (20 if big else max(1000, len(ds.sets)))
+    r = measure(epilogue_step(ds), n, 3)
+    us = timed(r, device) * 1e3 / n
+    fstep, plan = floor_step(w0.T, w0.H, 0)
+    fr = measure(fstep, n, 3)
+    floor_us = timed(fr, device) * 1e3 / n
+    gbs = w0.algorithmic_bytes() / (us * 1e-6) / 1e9
+    out = {"workload": name, "T": w0.T, "H": w0.H, "flags": flag_names(w0.flags),
+           "mode": "split" if plan.mode == E.MLA_MODE_SPLIT else "rows",
+           "bytes_per_call": w0.algorithmic_bytes(), "us_per_call": round(us, 3),
+           "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "launch_floor_us": round(floor_us, 3),
+           "floor_ratio": round(us / floor_us, 3), "calls": n, "sets": len(ds.sets),
+           "l2": f"{ds.touched / 2 ** 20:.0f} MiB touched per rotation"}
+    if w0.producer:
+        out.update(producer_pdl(ds, E, stream, device, n))
+    del r, fr
+    return out
+
+
+def producer_pdl(ds, E, stream, device, n):
+    """Producer alone vs producer + epilogue launched with PDL behind it."""
+    def prod(i):
+        d, _, (sn, sp) = ds.sets[i % len(ds.sets)]
+        rc = E.mla_harness_produce(sn.data_ptr(), sp.data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0),
+                                   d.q_nope.stride(1), d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1),
+                                   d.T, d.H, 0, stream.cuda_stream)
+        assert rc == E.MLA_OK
+
+    def pair(i):
+        prod(i)
+        d, q_out, _ = ds.sets[i % len(ds.sets)]
+        rc = E.launch_workload(d, q_out, extra_flags=E.MLA_FLAG_PDL, stream=stream)
+        assert rc == E.MLA_OK
+
+    def pair_nopdl(i):
+        prod(i)
+        d, q_out, _ = ds.sets[i % len(ds.sets)]
+        rc = E.launch_workload(d, q_out, stream=stream)
+        assert rc == E.MLA_OK
+
+    res = {}
+    for key, fn in (("producer_us", prod), ("producer_plus_epilogue_pdl_us", pair),
+                    ("producer_plus_epilogue_no_pdl_us", pair_nopdl)):
+        g = GraphRunner(fn, n, stream)
+        g.replay()
+        torch.cuda.synchronize()
+        res[key] = round(timed(g, device) * 1e3 / n, 3)
+        del g
+    res["epilogue_increment_pdl_us"] = round(res["producer_plus_epilogue_pdl_us"] - res["producer_us"], 3)
+    return res
+
+
+def run_e2e(args, w0, stream, device, world):
+    """Same metric through the user-facing call, with host buffers: every step
+    copies its inputs from pinned host memory, runs the epilogue and copies
+    q_out back, all on one stream, timed with CUDA events."""
+    from mla_decode_attention_10_b200 import epilogue as E
+    host = {k: getattr(w0, k).contiguous().pin_memory()
+            for k in ("q_nope", "q_pe", "kv_c", "k_pe", "slot_mapping", "positions")
+            if getattr(w0, k) is not None}
+    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    cache = w0.cache.to(device)
+    cos_sin = w0.cos_sin.to(device) if w0.cos_sin is not None else None
+    qs = w0.q_scale.to(device) if w0.q_scale is not None else None
+    ks = w0.kv_scale.to(device) if w0.kv_scale is not None else None
+    q_out = torch.empty((w0.T, w0.H, W.ROW), dtype=w0.q_out_dtype(), device=device)
+    q_host = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = q_host.numel() * q_host.element_size()
+
+    def step():
+        with torch.cuda.stream(stream):
+            for k, v in host.items():
+                dev[k].copy_(v, non_blocking=True)
+            E.fused_mla_decode_q_concat_kv_cache_insert(
+                dev["q_nope"], dev["q_pe"], dev["kv_c"], dev["k_pe"], cache, dev["slot_mapping"],
+                positions=dev.get("positions"), cos_sin=cos_sin, q_scale=qs, kv_scale=ks,
+                q_out=q_out, stream=stream)
+            q_host.copy_(q_out, non_blocking=True)
+
+    k = max(10, min(args.steps, 200))
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(k):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    ms = max_over_ranks(e0.elapsed_time(e1), device)
+    return {"value": round(job_us_per_call(ms, k, world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": k,
+            "path": "epilogue.fused_mla_decode_q_concat_kv_cache_insert, pinned host <-> device copies on the "
+                    "launch stream"}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle: the baseline and the reference arm
+# ---------------------------------------------------------------------------------------
+
+def _oracle_call(w):
+    import oracle
+    return oracle.run(w.q_nope, w.q_pe, w.kv_c, w.k_pe, w.slot_mapping, w.cache, w.flags,
+                      positions=w.positions, cos_sin=w.cos_sin, q_scale=w.q_scale, kv_scale=w.kv_scale)
+
+
+def cpu_baseline(name: str, seconds: float = 10.0):
+    """The single-threaded CPU oracle, as it stands, repeated on the workload
+    for about `seconds` of host time."""
+    w = named_variant(name, 0)
+    _oracle_call(w)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        _oracle_call(w)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(dt / n * 1e6, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} calls of {name} (T={w.T}, H={w.H}) in {dt:.1f} s, one host thread "
+                      f"({os.cpu_count()} cores on the host)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = named_variant(args.workload, 0)
+    for _ in range(args.warmup):
+        _oracle_call(w)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_call(w)
+    dt = time.perf_counter() - t0
+    us = dt / args.steps * 1e6
+    cb = {"value": round(us, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+          "sample": f"{args.steps} calls of {args.workload} (T={w.T}, H={w.H}), one host thread"}
+    return {"impl": "reference", "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "T": w.T, "H": w.H, "flags": flag_names(w.flags),
+                       "recipe": w.recipe, "implementation": "CPU oracle (oracle/mla_oracle.cpp)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(us, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------------------
+
+def parse(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default=HEADLINE, choices=W.names())
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be at least 3")
+    if a.steps < 1:
+        p.error("--steps must be positive")
+    return a
+
+
+def main(argv=None):
+    args = parse(argv)
+    rank, world, local_rank = rank_info()
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,62 @@
+/*
+ * mla_harness.h -- measurement and self-check kernels that sit beside the
+ * fused MLA decode epilogue (same library as mla_epilogue.h, same
+ * conventions: device pointers owned by the caller, asynchronous on
+ * `stream`, nothing allocated, host argument errors returned as mla_status).
+ *
+ * None of these is part of the epilogue itself; they exist to put it in the
+ * setting the vLLM PR #54896 report describes (an upstream producer kernel
+ * linked by programmatic dependent launch, 实现拆解 item 2), to time a bare
+ * launch, and to check the e4m3 quotient on the device.
+ */
+#ifndef MLA_HARNESS_H
+#define MLA_HARNESS_H
+
+#include <stdint.h>
+
+#include "mla_epilogue.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Synthetic upstream producer: writes q_nope [T,H,512] and q_pe [T,H,64]
+ * (bf16, strides as in mla_epilogue_launch) by copying src_nope [T,H,512] and
+ * src_pe [T,H,64] (contiguous bf16), standing in for the projection GEMM
+ * that produces the latent query (PR #54896 report, 实现拆解 item 2: the
+ * epilogue sits between an upstream GEMM and the attention kernel).  Each of
+ * its blocks signals griddepcontrol.launch_dependents when it starts, so a
+ * dependent launched with MLA_FLAG_PDL can be scheduled while it runs; the
+ * dependent's griddepcontrol.wait still waits for all of its stores.
+ * flags: MLA_FLAG_PDL (this launch itself is a programmatic dependent) only.
+ * Alignment: every pointer 16 bytes, strides multiples of 8 elements.
+ */
+MLA_API mla_status mla_harness_produce(const void* src_nope, const void* src_pe,
+                               void* q_nope, int64_t q_nope_stride_t, int64_t q_nope_stride_h,
+                               void* q_pe, int64_t q_pe_stride_t, int64_t q_pe_stride_h,
+                               int64_t T, int64_t H, uint32_t flags, mla_stream_t stream);
+
+/*
+ * An empty kernel launched with `blocks` x `threads` and, with MLA_FLAG_PDL,
+ * the programmatic-serialization attribute: the bare-launch floor that the
+ * epilogue's latency at decode sizes is compared with.
+ */
+MLA_API mla_status mla_harness_empty(int64_t blocks, int32_t threads, uint32_t flags, mla_stream_t stream);
+
+/*
+ * Device check of the e4m3 quotient: for every fp32 bit pattern p in
+ * [first, first + count) compares the epilogue's quotient x / scale with the
+ * CUDA IEEE division __fdiv_rn (NaN equal to NaN) and the e4m3 bytes they
+ * encode to.  result (device, 3 x uint64, overwritten): [0] quotients that
+ * differ, [1] e4m3 bytes that differ, [2] smallest differing pattern
+ * (UINT64_MAX if none).  first + count <= 2^32.
+ */
+MLA_API mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t count,
+                                 unsigned long long* result, mla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_HARNESS_H */

@@ -1,0 +1,150 @@
+// mla_harness.cu -- synthetic producer, bare-launch kernel and quotient self-check
+// that sit beside the epilogue (declarations and contracts in mla_harness.h).
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "latent_math.cuh"
+#include "mla_harness.h"
+
+namespace mla {
+namespace harness {
+
+// One warp per (token, head) row: 1024 bytes of nope (two 16-byte chunks per
+// lane) and 128 bytes of pe (lanes 0..7), grid-stride.
+__global__ void __launch_bounds__(256) produce_kernel(const uint4* __restrict__ src_nope,
+                                                      const uint4* __restrict__ src_pe,
+                                                      uint16_t* q_nope, int64_t qn_st, int64_t qn_sh,
+                                                      uint16_t* q_pe, int64_t qp_st, int64_t qp_sh,
+                                                      int64_t T, int64_t H) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t rows = T * H;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += warps) {
+    const int64_t t = r / H;
+    const int64_t h = r - t * H;
+    const uint4 a = src_nope[r * 64 + lane];
+    const uint4 b = src_nope[r * 64 + 32 + lane];
+    uint4 p = make_uint4(0, 0, 0, 0);
+    if (lane < 8) p = src_pe[r * 8 + lane];
+    uint4* dn = reinterpret_cast<uint4*>(q_nope + t * qn_st + h * qn_sh);
+    dn[lane] = a;
+    dn[32 + lane] = b;
+    if (lane < 8) reinterpret_cast<uint4*>(q_pe + t * qp_st + h * qp_sh)[lane] = p;
+  }
+}
+
+__global__ void empty_kernel() {}
+
+__global__ void __launch_bounds__(256) div_check_kernel(float scale, uint64_t first, uint64_t count,
+                                                        unsigned long long* result) {
+  const Divisor d = make_divisor(scale);
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  unsigned long long bad_q = 0, bad_b = 0, lowest = ~0ull;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
+    const uint64_t p = first + i;
+    const float x = __uint_as_float(static_cast<uint32_t>(p));
+    const float q = div_rn(x, d);
+    const float ref = __fdiv_rn(x, scale);
+    const bool same_q = (__float_as_uint(q) == __float_as_uint(ref)) || (isnan(q) && isnan(ref));
+    const uint32_t bq = pack_e4m3x2(q, 0.0f) & 0xffu;
+    const uint32_t br = pack_e4m3x2(ref, 0.0f) & 0xffu;
+    if (!same_q) {
+      ++bad_q;
+      if (p < lowest) lowest = p;
+    }
+    if (bq != br) {
+      ++bad_b;
+      if (p < lowest) lowest = p;
+    }
+  }
+  if (bad_q) atomicAdd(result + 0, bad_q);
+  if (bad_b) atomicAdd(result + 1, bad_b);
+  if (lowest != ~0ull) atomicMin(result + 2, lowest);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mla_status finish(cudaError_t e) {
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+mla_status launch(const void* fn, dim3 grid, dim3 block, bool pdl, cudaStream_t stream, void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return finish(cudaLaunchKernelExC(&cfg, fn, args));
+}
+
+}  // namespace harness
+}  // namespace mla
+
+extern "C" {
+
+mla_status mla_harness_produce(const void* src_nope, const void* src_pe, void* q_nope, int64_t q_nope_stride_t,
+                               int64_t q_nope_stride_h, void* q_pe, int64_t q_pe_stride_t, int64_t q_pe_stride_h,
+                               int64_t T, int64_t H, uint32_t flags, mla_stream_t stream) {
+  using namespace mla::harness;
+  if ((flags & ~MLA_FLAG_PDL) != 0) return MLA_ERR_UNSUPPORTED;
+  if (T < 0 || H < 1 || T > (INT64_C(1) << 31) / H) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!src_nope || !src_pe || !q_nope || !q_pe) return MLA_ERR_INVALID_ARG;
+  if (q_nope_stride_t < 0 || q_nope_stride_h < 0 || q_pe_stride_t < 0 || q_pe_stride_h < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(src_nope) || !aligned16(src_pe) || !aligned16(q_nope) || !aligned16(q_pe) ||
+      (q_nope_stride_t % 8) || (q_nope_stride_h % 8) || (q_pe_stride_t % 8) || (q_pe_stride_h % 8))
+    return MLA_ERR_ALIGNMENT;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return finish(cudaErrorUnknown);
+  const int64_t rows = T * H;
+  int64_t blocks = (rows + 7) / 8;
+  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  const uint4* sn = static_cast<const uint4*>(src_nope);
+  const uint4* sp = static_cast<const uint4*>(src_pe);
+  uint16_t* qn = static_cast<uint16_t*>(q_nope);
+  uint16_t* qp = static_cast<uint16_t*>(q_pe);
+  void* args[] = {&sn, &sp, &qn, &q_nope_stride_t, &q_nope_stride_h, &qp, &q_pe_stride_t, &q_pe_stride_h, &T, &H};
+  return launch(reinterpret_cast<const void*>(&produce_kernel), dim3(static_cast<unsigned>(blocks)), dim3(256),
+                (flags & MLA_FLAG_PDL) != 0, reinterpret_cast<cudaStream_t>(stream), args);
+}
+
+mla_status mla_harness_empty(int64_t blocks, int32_t threads, uint32_t flags, mla_stream_t stream) {
+  using namespace mla::harness;
+  if ((flags & ~MLA_FLAG_PDL) != 0) return MLA_ERR_UNSUPPORTED;
+  if (blocks < 1 || blocks > INT32_MAX || threads < 1 || threads > 1024) return MLA_ERR_INVALID_ARG;
+  return launch(reinterpret_cast<const void*>(&empty_kernel), dim3(static_cast<unsigned>(blocks)),
+                dim3(static_cast<unsigned>(threads)), (flags & MLA_FLAG_PDL) != 0,
+                reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t count, unsigned long long* result,
+                                 mla_stream_t stream) {
+  using namespace mla::harness;
+  if (result == nullptr || (reinterpret_cast<uintptr_t>(result) & 7u) != 0) return MLA_ERR_INVALID_ARG;
+  if (first > (UINT64_C(1) << 32) || count > (UINT64_C(1) << 32) - first) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(result, 0, 2 * sizeof(unsigned long long), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(result + 2, 0xff, sizeof(unsigned long long), s);
+  if (e != cudaSuccess) return finish(e);
+  if (count == 0) return MLA_OK;
+  void* args[] = {&scale, &first, &count, &result};
+  return launch(reinterpret_cast<const void*>(&div_check_kernel), dim3(148 * 16), dim3(256), false, s, args);
+}
+
+}  // extern "C"

@@ -16,7 +16,7 @@ batch behind a synthetic producer.
 from __future__ import annotations
 
 import dataclasses
-import math
+import functools
 from typing import Dict, List, Optional
 
 import numpy as np
@@ -105,15 +105,22 @@ def _move(v: torch.Tensor, device) -> torch.Tensor:
     return nb.as_strided(v.size(), v.stride(), v.storage_offset())
 
 
-def rope_table(rows: int, base: float = ROPE_BASE) -> torch.Tensor:
-    """fp32 [rows, 64] table: row p = [cos(p*w_0..31) | sin(p*w_0..31)],
-    w_j = base^(-j/32) (rotate-half frequencies for 64 rotary dims),
-    evaluated in double precision and rounded once to fp32."""
+@functools.lru_cache(maxsize=4)
+def _rope_table_np(rows: int, base: float) -> np.ndarray:
     p = np.arange(rows, dtype=np.float64)[:, None]
     w = base ** (-np.arange(PE // 2, dtype=np.float64) / (PE // 2))
     ang = p * w[None, :]
     tab = np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(np.float32)
-    return torch.from_numpy(np.ascontiguousarray(tab))
+    tab.setflags(write=False)
+    return tab
+
+
+def rope_table(rows: int, base: float = ROPE_BASE) -> torch.Tensor:
+    """fp32 [rows, 64] table: row p = [cos(p*w_0..31) | sin(p*w_0..31)],
+    w_j = base^(-j/32) (rotate-half frequencies for 64 rotary dims),
+    evaluated in double precision and rounded once to fp32 (a fresh copy
+    per call)."""
+    return torch.from_numpy(np.array(_rope_table_np(rows, base), copy=True))
 
 
 def _randn_bf16(g: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
@@ -176,56 +183,74 @@ def make(name: str, T: int, H: int, flags: int, *, seed: int, num_blocks: int,
 
 # --- the named workloads -------------------------------------------------------------
 
+DECODE_SWEEP_T = (1, 2, 4, 8, 16, 32, 64, 128, 256)
+_ALL_FP8 = FLAG_ROPE | FLAG_Q_FP8 | FLAG_KV_FP8
+
+
+def _recipes() -> Dict[str, dict]:
+    r = {
+        "decode_t4_h16": dict(
+            T=4, H=16, flags=0, seed=0, num_blocks=1,
+            recipe="T=4 H=16 bf16 N(0,1), no RoPE/FP8, zero cache [1,64,576], slots randperm(64)[:4], seed 0"),
+    }
+    for T in (64, 65):
+        r[f"split_boundary_t{T}_h16_rope"] = dict(
+            T=T, H=16, flags=FLAG_ROPE, seed=3, num_blocks=2, rope_rows=32768,
+            recipe=f"T={T} H=16 bf16 N(0,1), RoPE (32768-row table, positions U[0,32768)), "
+                   "zero cache [2,64,576], slots randperm(128)[:T], seed 3")
+    for T in DECODE_SWEEP_T:
+        r[f"decode_sweep_t{T}_h16_rope_fp8"] = dict(
+            T=T, H=16, flags=_ALL_FP8, seed=0, num_blocks=4096, std=2.0, rope_rows=32768, scale=0.05,
+            cache_fill="random",
+            recipe=f"T={T} H=16 bf16 N(0,2), RoPE, Q/KV e4m3 scale 0.05, random-byte e4m3 cache "
+                   "[4096,64,576], slots randperm(262144)[:T], seed 0")
+    r["prefill_t1024_h128_strided"] = dict(
+        T=1024, H=128, flags=FLAG_ROPE, seed=0, num_blocks=1024, rope_rows=32768, q_nope_row=640,
+        kv_c_row=1536, kv_c_offset=512,
+        recipe="T=1024 H=128 bf16 N(0,1), RoPE; q_nope = [1024,128,640][:,:,:512], "
+               "kv_c = [1024,1536][:,512:1024]; zero cache [1024,64,576]; slots randperm(65536)[:1024], seed 0")
+    r["batch_t8192_h16_pdl_fp8"] = dict(
+        T=8192, H=16, flags=_ALL_FP8, seed=0, num_blocks=16384, rope_rows=131072, scale=0.05,
+        cache_fill="random", producer=True,
+        recipe="T=8192 H=16 bf16 N(0,1), RoPE (131072-row table), Q/KV e4m3 scale 0.05, random-byte e4m3 "
+               "cache [16384,64,576], slots randperm(1048576)[:8192], q_nope/q_pe written by a producer "
+               "kernel, epilogue launched with PDL, seed 0")
+    return r
+
+
+RECIPES = _recipes()
+
+
+def named(name: str, seed_offset: int = 0) -> Workload:
+    """The named workload; ``seed_offset`` draws fresh values of the same recipe."""
+    kw = dict(RECIPES[name])
+    kw["seed"] += seed_offset
+    return make(name, **kw)
+
+
 def decode_t4_h16() -> Workload:
-    return make("decode_t4_h16", 4, 16, 0, seed=0, num_blocks=1,
-                recipe="T=4 H=16 bf16 N(0,1), no RoPE/FP8, zero cache [1,64,576], slots randperm(64)[:4], seed 0")
+    return named("decode_t4_h16")
 
 
 def split_boundary(T: int) -> Workload:
-    assert T in (64, 65)
-    return make(f"split_boundary_t{T}_h16_rope", T, 16, FLAG_ROPE, seed=3, num_blocks=2,
-                rope_rows=32768,
-                recipe=f"T={T} H=16 bf16 N(0,1), RoPE (32768-row table, positions U[0,32768)), "
-                       "zero cache [2,64,576], slots randperm(128)[:T], seed 3")
-
-
-DECODE_SWEEP_T = (1, 2, 4, 8, 16, 32, 64, 128, 256)
+    return named(f"split_boundary_t{T}_h16_rope")
 
 
 def decode_sweep(T: int) -> Workload:
-    return make(f"decode_sweep_t{T}_h16_rope_fp8", T, 16, FLAG_ROPE | FLAG_Q_FP8 | FLAG_KV_FP8,
-                seed=0, num_blocks=4096, std=2.0, rope_rows=32768, scale=0.05, cache_fill="random",
-                recipe=f"T={T} H=16 bf16 N(0,2), RoPE, Q/KV e4m3 scale 0.05, random-byte e4m3 cache "
-                       "[4096,64,576], slots randperm(262144)[:T], seed 0")
+    return named(f"decode_sweep_t{T}_h16_rope_fp8")
 
 
 def prefill_t1024_h128_strided() -> Workload:
-    return make("prefill_t1024_h128_strided", 1024, 128, FLAG_ROPE, seed=0, num_blocks=1024,
-                rope_rows=32768, q_nope_row=640, kv_c_row=1536, kv_c_offset=512,
-                recipe="T=1024 H=128 bf16 N(0,1), RoPE; q_nope = [1024,128,640][:,:,:512], "
-                       "kv_c = [1024,1536][:,512:1024]; zero cache [1024,64,576]; "
-                       "slots randperm(65536)[:1024], seed 0")
+    return named("prefill_t1024_h128_strided")
 
 
 def batch_t8192_h16_pdl_fp8() -> Workload:
-    return make("batch_t8192_h16_pdl_fp8", 8192, 16, FLAG_ROPE | FLAG_Q_FP8 | FLAG_KV_FP8,
-                seed=0, num_blocks=16384, rope_rows=131072, scale=0.05, cache_fill="random",
-                producer=True,
-                recipe="T=8192 H=16 bf16 N(0,1), RoPE (131072-row table), Q/KV e4m3 scale 0.05, "
-                       "random-byte e4m3 cache [16384,64,576], slots randperm(1048576)[:8192], "
-                       "q_nope/q_pe written by a producer kernel, epilogue launched with PDL, seed 0")
+    return named("batch_t8192_h16_pdl_fp8")
 
 
 def all_named() -> Dict[str, "callable"]:
-    d = {"decode_t4_h16": decode_t4_h16,
-         "split_boundary_t64_h16_rope": lambda: split_boundary(64),
-         "split_boundary_t65_h16_rope": lambda: split_boundary(65)}
-    for t in DECODE_SWEEP_T:
-        d[f"decode_sweep_t{t}_h16_rope_fp8"] = (lambda tt: (lambda: decode_sweep(tt)))(t)
-    d["prefill_t1024_h128_strided"] = prefill_t1024_h128_strided
-    d["batch_t8192_h16_pdl_fp8"] = batch_t8192_h16_pdl_fp8
-    return d
+    return {n: (lambda nn: (lambda: named(nn)))(n) for n in RECIPES}
 
 
 def names() -> List[str]:
-    return list(all_named().keys())
+    return list(RECIPES.keys())

@@ -1,0 +1,189 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the
+headers declare, agrees with the binding's constants, and rejects bad host
+arguments before it makes any CUDA call."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from mla_decode_attention_10_b200 import build as B
+from mla_decode_attention_10_b200 import epilogue as E
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("mla_epilogue.h", "mla_harness.h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return E.lib()
+
+
+def _declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        names += re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", text)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 9
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+    # nothing else leaks out of the library
+    ours = {n for n in exported if n.startswith("mla_")}
+    assert ours == set(names)
+
+
+def test_header_constants_match_binding():
+    text = "".join(open(h).read() for h in HEADERS)
+    defines = dict(re.findall(r"#define\s+(MLA_\w+)\s+(\d+)u?", text))
+    enums = dict(re.findall(r"(MLA_(?:OK|ERR_\w+))\s*=\s*(\d+)", text))
+    for name, val in list(defines.items()) + list(enums.items()):
+        assert getattr(E, name) == int(val), name
+
+
+def test_oracle_and_binding_flags_agree():
+    import oracle
+    from mla_decode_attention_10_b200 import workloads as W
+    assert oracle.FLAG_ROPE == W.FLAG_ROPE == E.MLA_FLAG_ROPE
+    assert oracle.FLAG_Q_FP8 == W.FLAG_Q_FP8 == E.MLA_FLAG_Q_FP8
+    assert oracle.FLAG_KV_FP8 == W.FLAG_KV_FP8 == E.MLA_FLAG_KV_FP8
+    assert W.FLAG_PDL == E.MLA_FLAG_PDL
+    assert oracle.STATUS_SLOT_RANGE == E.MLA_STATUS_SLOT_RANGE
+    assert oracle.STATUS_POS_RANGE == E.MLA_STATUS_POS_RANGE
+
+
+# Fake, well-aligned addresses: every call below must return before touching them.
+A = 1 << 20
+
+
+def _call(**kw):
+    args = dict(q_nope=A, q_nope_stride_t=16 * 512, q_nope_stride_h=512, q_pe=A, q_pe_stride_t=16 * 64,
+                q_pe_stride_h=64, kv_c=A, kv_c_stride_t=512, k_pe=A, k_pe_stride_t=64, slot_mapping=A,
+                positions=A, cos_sin=A, rope_rows=8, q_scale=A, kv_scale=A, T=4, H=16, block_size=64,
+                num_blocks=1, flags=0, q_out=A, cache=A, status=None, stream=None)
+    args.update(kw)
+    return E.mla_epilogue_launch(**args)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(flags=64), E.MLA_ERR_UNSUPPORTED),
+    (dict(flags=1 << 31), E.MLA_ERR_UNSUPPORTED),
+    (dict(flags=E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS), E.MLA_ERR_INVALID_ARG),
+    (dict(T=-1), E.MLA_ERR_INVALID_ARG),
+    (dict(H=0), E.MLA_ERR_INVALID_ARG),
+    (dict(H=65537), E.MLA_ERR_INVALID_ARG),
+    (dict(block_size=0), E.MLA_ERR_INVALID_ARG),
+    (dict(num_blocks=-1), E.MLA_ERR_INVALID_ARG),
+    (dict(T=2 ** 31 // 17 + 1), E.MLA_ERR_INVALID_ARG),
+    (dict(q_nope=None), E.MLA_ERR_INVALID_ARG),
+    (dict(q_pe=None), E.MLA_ERR_INVALID_ARG),
+    (dict(kv_c=None), E.MLA_ERR_INVALID_ARG),
+    (dict(k_pe=None), E.MLA_ERR_INVALID_ARG),
+    (dict(slot_mapping=None), E.MLA_ERR_INVALID_ARG),
+    (dict(q_out=None), E.MLA_ERR_INVALID_ARG),
+    (dict(cache=None), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_ROPE, positions=None), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_ROPE, cos_sin=None), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_ROPE, rope_rows=0), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_Q_FP8, q_scale=None), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_KV_FP8, kv_scale=None), E.MLA_ERR_INVALID_ARG),
+    (dict(q_nope_stride_t=-8), E.MLA_ERR_INVALID_ARG),
+    (dict(k_pe_stride_t=-1), E.MLA_ERR_INVALID_ARG),
+    (dict(q_nope=A + 8), E.MLA_ERR_ALIGNMENT),
+    (dict(kv_c=A + 2), E.MLA_ERR_ALIGNMENT),
+    (dict(q_out=A + 4), E.MLA_ERR_ALIGNMENT),
+    (dict(cache=A + 8), E.MLA_ERR_ALIGNMENT),
+    (dict(q_nope_stride_t=16 * 512 + 4), E.MLA_ERR_ALIGNMENT),
+    (dict(q_nope_stride_h=516), E.MLA_ERR_ALIGNMENT),
+    (dict(kv_c_stride_t=520 + 2), E.MLA_ERR_ALIGNMENT),
+    (dict(q_pe=A + 1), E.MLA_ERR_ALIGNMENT),
+    (dict(k_pe=A + 1), E.MLA_ERR_ALIGNMENT),
+    (dict(slot_mapping=A + 4), E.MLA_ERR_ALIGNMENT),
+    (dict(flags=E.MLA_FLAG_ROPE, positions=A + 2), E.MLA_ERR_ALIGNMENT),
+    (dict(flags=E.MLA_FLAG_ROPE, cos_sin=A + 2), E.MLA_ERR_ALIGNMENT),
+    (dict(flags=E.MLA_FLAG_Q_FP8, q_scale=A + 1), E.MLA_ERR_ALIGNMENT),
+    (dict(status=A + 2), E.MLA_ERR_ALIGNMENT),
+])
+def test_host_validation_rejects_before_any_cuda_call(lib, kw, code):
+    assert _call(**kw) == code
+
+
+def test_zero_tokens_launches_nothing(lib):
+    # T == 0 returns OK even with null buffers: nothing is read or written
+    assert _call(T=0, q_nope=None, q_pe=None, kv_c=None, k_pe=None, slot_mapping=None,
+                 q_out=None, cache=None) == E.MLA_OK
+
+
+def test_size_one_dimensions_skip_stride_checks(lib):
+    # a stride of a size-1 dimension is never used, so it is not checked; the
+    # call then proceeds to the device query, which fails without a GPU
+    import torch
+    rc = _call(T=1, H=1, q_nope_stride_t=3, q_nope_stride_h=5, kv_c_stride_t=7)
+    assert rc in ((E.MLA_OK,) if torch.cuda.is_available() else (E.MLA_ERR_CUDA,))
+
+
+def test_plan_modes_and_grids(lib):
+    p = E.mla_epilogue_plan(64, 16, 0, sm_count=148)
+    assert p.mode == E.MLA_MODE_SPLIT and p.threads_per_block == 96 * p.rows_per_block
+    assert p.blocks == -(-64 * 17 // p.rows_per_block)
+    p = E.mla_epilogue_plan(65, 16, 0, sm_count=148)
+    assert p.mode == E.MLA_MODE_ROWS and p.threads_per_block % 32 == 0
+    assert p.blocks <= 148 * E.mla_epilogue_get_tuning().rows_blocks_per_sm
+    assert p.blocks % 148 == 0 or p.blocks * (p.threads_per_block // 32) >= 65 * 17
+    assert E.mla_epilogue_plan(1, 16, E.MLA_FLAG_FORCE_ROWS, sm_count=148).mode == E.MLA_MODE_ROWS
+    assert E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148).mode == E.MLA_MODE_SPLIT
+    big = E.mla_epilogue_plan(8192, 16, 0, sm_count=148)
+    assert big.blocks == 148 * E.mla_epilogue_get_tuning().rows_blocks_per_sm
+    with pytest.raises(E.MlaError):
+        E.mla_epilogue_plan(0, 16, 0, sm_count=148)
+    with pytest.raises(E.MlaError):
+        E.mla_epilogue_plan(4, 16, E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS, sm_count=148)
+
+
+def test_tuning_moves_the_threshold_and_clamps(lib):
+    old = E.mla_epilogue_get_tuning()
+    try:
+        E.mla_epilogue_set_tuning(split_max_tokens=128)
+        assert E.mla_epilogue_plan(100, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
+        E.mla_epilogue_set_tuning(split_rows_per_block=99, rows_warps_per_block=99, rows_blocks_per_sm=99)
+        t = E.mla_epilogue_get_tuning()
+        assert t.split_rows_per_block == 4 and t.rows_warps_per_block == 8 and t.rows_blocks_per_sm <= 5
+        E.mla_epilogue_set_tuning()  # all zero: unchanged
+        assert E.mla_epilogue_get_tuning().split_max_tokens == 128
+    finally:
+        E.mla_epilogue_set_tuning(old.split_max_tokens, old.split_rows_per_block,
+                                  old.rows_warps_per_block, old.rows_blocks_per_sm)
+
+
+def test_status_strings(lib):
+    for c in range(5):
+        assert E.status_string(c).startswith("MLA_")
+    assert "unknown" in E.status_string(99)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(flags=1), E.MLA_ERR_UNSUPPORTED),
+    (dict(T=-1), E.MLA_ERR_INVALID_ARG),
+    (dict(src_nope=None), E.MLA_ERR_INVALID_ARG),
+    (dict(q_nope=A + 8), E.MLA_ERR_ALIGNMENT),
+    (dict(q_pe_stride_h=65), E.MLA_ERR_ALIGNMENT),
+])
+def test_harness_validation(lib, kw, code):
+    args = dict(src_nope=A, src_pe=A, q_nope=A, q_nope_stride_t=16 * 512, q_nope_stride_h=512, q_pe=A,
+                q_pe_stride_t=16 * 64, q_pe_stride_h=64, T=4, H=16, flags=0, stream=None)
+    args.update(kw)
+    assert E.mla_harness_produce(**args) == code
+    assert E.mla_harness_empty(0, 32, 0, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_empty(1, 2048, 0, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_div_check(1.0, 0, 2 ** 32 + 1, A, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_div_check(1.0, 0, 1, None, None) == E.MLA_ERR_INVALID_ARG
