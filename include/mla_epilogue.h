@@ -92,9 +92,11 @@ typedef enum mla_status {
  *            that token's rows unrotated and sets MLA_STATUS_POS_RANGE.
  *   q_scale, kv_scale  one fp32 each in device memory (read by the kernel, so
  *            an upstream kernel may write them); read only with the matching
- *            FP8 flag (may be NULL otherwise).  Any positive finite scale
- *            gives the exact IEEE quotient; other values give whatever
- *            x / scale gives in IEEE arithmetic.
+ *            FP8 flag (may be NULL otherwise).  For any scale the e4m3
+ *            byte is that of the IEEE fp32 quotient x / scale (the kernel
+ *            computes that quotient bit for bit whenever |x| >= 2^-100 and
+ *            |x / scale| < 2^125; outside, both round to the same signed
+ *            zero or to +-448).
  *   T >= 0 tokens (T == 0: nothing is launched, MLA_OK); H >= 1 heads;
  *   block_size >= 1, num_blocks >= 0: cache geometry.
  *   q_out    [T, H, 576] contiguous; bf16, or e4m3 bytes with MLA_FLAG_Q_FP8.

@@ -48,9 +48,12 @@ MLA_API mla_status mla_harness_empty(int64_t blocks, int32_t threads, uint32_t f
  * Device check of the e4m3 quotient: for every fp32 bit pattern p in
  * [first, first + count) compares the epilogue's quotient x / scale with the
  * CUDA IEEE division __fdiv_rn (NaN equal to NaN) and the e4m3 bytes they
- * encode to.  result (device, 3 x uint64, overwritten): [0] quotients that
- * differ, [1] e4m3 bytes that differ, [2] smallest differing pattern
- * (UINT64_MAX if none).  first + count <= 2^32.
+ * encode to.  result (device, 3 x uint64, overwritten): [0] inputs with
+ * |x| >= 2^-100 and |x / scale| < 2^125 whose quotients differ (outside that
+ * range the epilogue's quotient may differ in its last bits while its e4m3
+ * byte, a signed zero below and +-448 above, may not), [1] inputs whose e4m3
+ * bytes differ, [2] smallest pattern counted in [0] or [1] (UINT64_MAX if
+ * none).  first + count <= 2^32.
  */
 MLA_API mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t count,
                                  unsigned long long* result, mla_stream_t stream);

@@ -69,11 +69,13 @@ __device__ __forceinline__ Divisor make_divisor(float s) {
 // one fused multiply-add whenever q is within an ulp of x/s, and
 // RN(q + r y) is then the correctly rounded quotient.  q0 = RN(x y) can be
 // up to ~1.5 ulp off, so one correction step first makes it faithful, and a
-// second one rounds it correctly.  Zero keeps the sign of x (s > 0); when
-// |x y| is not below 2^100 (huge, infinite or NaN input) the e4m3 result
-// saturates or is NaN whatever the last bits are, so q0 is returned as is.
-// Below |x| ~ 2^-102 the residual may underflow, but there |x / s| <= 2^-38,
-// which every e4m3 rounding sends to a signed zero.
+// second one rounds it correctly.  Zero keeps the sign of x (s > 0).  When
+// |x y| is not below 2^126 (so that no correction step could overflow) or is
+// infinite or NaN, q0 is returned as is: the e4m3 result saturates to 448 or
+// is NaN whatever its last bits are.
+// Below |x| ~ 2^-102 the residual may underflow and the last bits of the
+// quotient may then differ from the IEEE quotient, but there |x / s| <= 2^-38,
+// which every e4m3 rounding sends to the same signed zero.
 __device__ __forceinline__ float div_rn(float x, const Divisor& d) {
   if (!d.fast) return __fdiv_rn(x, d.s);
   const float q0 = __fmul_rn(x, d.y);
@@ -81,7 +83,7 @@ __device__ __forceinline__ float div_rn(float x, const Divisor& d) {
   const float q1 = __fmaf_rn(r0, d.y, q0);
   const float r1 = __fmaf_rn(-q1, d.s, x);
   const float q2 = __fmaf_rn(r1, d.y, q1);
-  return fabsf(q0) < 0x1p100f ? copysignf(q2, x) : q0;
+  return fabsf(q0) < 0x1p126f ? copysignf(q2, x) : q0;
 }
 
 // Eight bf16 (one 16-byte chunk) -> eight e4m3 bytes of x / s.

@@ -110,7 +110,8 @@ DIV_SCALES = [0.05, 1.0, 0.37, 3.0, 7.0, 0.9, 1.0 / 3.0, 2.0 ** -64, 2.0 ** 64, 
 @pytest.mark.parametrize("scale", DIV_SCALES)
 def test_quotient_equals_ieee_division_for_every_fp32(scale):
     """The epilogue's x / scale against CUDA's IEEE division for all 2^32 fp32
-    bit patterns: same quotient bits and same e4m3 byte, NaN counted equal."""
+    bit patterns: the same e4m3 byte everywhere, and the same quotient bits
+    for 2^-100 <= |x| and |x / scale| < 2^125 (NaN counted equal)."""
     res = torch.zeros(3, dtype=torch.int64, device="cuda")
     rc = E.mla_harness_div_check(scale, 0, 2 ** 32, res.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert rc == E.MLA_OK
@@ -127,7 +128,7 @@ def test_zero_tokens_touches_nothing():
     before = d.cache.clone()
     assert E.launch_workload(d, q) == E.MLA_OK
     torch.cuda.synchronize()
-    assert torch.equal(d.cache, before)
+    assert torch.equal(d.cache.view(torch.int16), before.view(torch.int16))
 
 
 @pytest.mark.parametrize("force", FORCE)
@@ -172,7 +173,7 @@ def test_misaligned_arguments_launch_nothing():
         args[k] += off
         assert E.mla_epilogue_launch(**args) == E.MLA_ERR_ALIGNMENT
     torch.cuda.synchronize()
-    assert torch.equal(d.cache, before) and torch.count_nonzero(q) == 0
+    assert torch.equal(d.cache.view(torch.int16), before.view(torch.int16)) and torch.count_nonzero(q) == 0
     assert E.mla_epilogue_launch(**base) == E.MLA_OK
     torch.cuda.synchronize()
     assert torch.count_nonzero(q) > 0
