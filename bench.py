@@ -191,10 +191,11 @@ class GraphRunner:
             g.replay()
 
 
-def timed(runner: GraphRunner, device) -> float:
+def timed(runner: GraphRunner, device, flush: bool = True) -> float:
     """ms for one replay of all graphs, bracketed by barrier + synchronize, max over ranks."""
     s = runner.stream
-    flush_l2()
+    if flush:
+        flush_l2()
     barrier(device)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -313,9 +314,9 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.Stream(device)
     peak, peak_note = measured_hbm_gbs()
 
-    def epilogue_step(ds, extra=0):
+    def epilogue_step(ds, extra=0, single_set=False):
         def f(i):
-            d, q_out, _ = ds.sets[i % len(ds.sets)]
+            d, q_out, _ = ds.sets[0 if single_set else i % len(ds.sets)]
             rc = E.launch_workload(d, q_out, extra_flags=extra, stream=stream)
             if rc != E.MLA_OK:
                 raise E.MlaError(rc, "mla_epilogue_launch")
@@ -377,6 +378,14 @@ def run_ours(args, rank, world, local_rank):
     pdl_floor_us = timed(pfrunner, device) * 1e3 / args.steps
     del prunner, pfrunner
 
+    # same inputs every call: they stay in L2, as when the upstream kernel has just written them
+    wrunner = measure(epilogue_step(ds, 0, single_set=True), args.steps, args.warmup)
+    warm_us = timed(wrunner, device, flush=False) * 1e3 / args.steps
+    del wrunner
+
+    # producer -> epilogue -> consumer, with and without programmatic dependent launch
+    chain = producer_consumer_chain(ds, E, stream, device, min(args.steps, 500), args.warmup)
+
     # ---- end to end through the Python API: pinned host inputs -> call -> q_out to host
     e2e = run_e2e(args, w0, stream, device, world)
 
@@ -402,7 +411,12 @@ def run_ours(args, rank, world, local_rank):
         "launch_floor_us": round(floor_us, 4),
         "floor_ratio": round(per_call_us_rank / floor_us, 3),
         "pdl_chain": {"us_per_call": round(pdl_us, 4), "floor_us": round(pdl_floor_us, 4),
-                      "floor_ratio": round(pdl_us / pdl_floor_us, 3)},
+                      "floor_ratio": round(pdl_us / pdl_floor_us, 3),
+                      "note": "each call a programmatic dependent of the previous one (disjoint input sets)"},
+        "l2_warm": {"us_per_call": round(warm_us, 4), "floor_ratio": round(warm_us / floor_us, 3),
+                    "note": "the same inputs every call, so they are L2-resident (not the headline: the "
+                            "headline reads HBM)"},
+        "producer_epilogue_consumer": chain,
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "traffic": None,
                      "peak_source": peak_note,
@@ -485,6 +499,49 @@ def producer_pdl(ds, E, stream, device, n):
         del g
     res["epilogue_increment_pdl_us"] = round(res["producer_plus_epilogue_pdl_us"] - res["producer_us"], 3)
     return res
+
+
+def producer_consumer_chain(ds, E, stream, device, n, warmup):
+    """Per step: the synthetic producer writes a set's q_nope / q_pe, the
+    epilogue runs on that set, and the synthetic consumer reads its q_out and
+    cache rows.  Timed with the epilogue and the consumer launched as
+    programmatic dependents (PDL) and without; `producer_us` alone for
+    reference.  Values do not matter here (the producer copies the next
+    set's query inputs); stream order keeps every step after the last."""
+    S = len(ds.sets)
+    w0 = ds.w0
+    scores = torch.empty(w0.T * w0.H, dtype=torch.float32, device=device)
+    cflags = (E.MLA_FLAG_Q_FP8 if w0.q_fp8 else 0) | (E.MLA_FLAG_KV_FP8 if w0.kv_fp8 else 0)
+
+    def prod(i):
+        d, _, src = ds.sets[i % S]
+        sn, sp = src if src is not None else (ds.sets[(i + 1) % S][0].q_nope, ds.sets[(i + 1) % S][0].q_pe)
+        assert sn.is_contiguous() and sp.is_contiguous()
+        rc = E.mla_harness_produce(sn.data_ptr(), sp.data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0),
+                                   d.q_nope.stride(1), d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1),
+                                   d.T, d.H, 0, stream.cuda_stream)
+        assert rc == E.MLA_OK
+
+    def chain(pdl):
+        def f(i):
+            prod(i)
+            d, q_out, _ = ds.sets[i % S]
+            assert E.launch_workload(d, q_out, extra_flags=pdl, stream=stream) == E.MLA_OK
+            assert E.mla_harness_consume(q_out.data_ptr(), d.cache.data_ptr(), d.slot_mapping.data_ptr(), d.T, d.H,
+                                         d.num_blocks * d.block_size, cflags | pdl, scores.data_ptr(),
+                                         stream.cuda_stream) == E.MLA_OK
+        return f
+
+    out = {}
+    for key, fn in (("producer_us", prod), ("chain_pdl_us", chain(E.MLA_FLAG_PDL)), ("chain_no_pdl_us", chain(0))):
+        g = GraphRunner(fn, n, stream)
+        g.replay()
+        torch.cuda.synchronize()
+        out[key] = round(timed(g, device) * 1e3 / n, 3)
+        del g
+    out["pdl_saves_us"] = round(out["chain_no_pdl_us"] - out["chain_pdl_us"], 3)
+    out["steps"] = n
+    return out
 
 
 def run_e2e(args, w0, stream, device, world):

@@ -95,7 +95,7 @@ typedef enum mla_status {
  *            FP8 flag (may be NULL otherwise).  For any scale the e4m3
  *            byte is that of the IEEE fp32 quotient x / scale (the kernel
  *            computes that quotient bit for bit whenever |x| >= 2^-100 and
- *            |x / scale| < 2^125; outside, both round to the same signed
+ *            |x / scale| < 448; outside, both round to the same signed
  *            zero or to +-448).
  *   T >= 0 tokens (T == 0: nothing is launched, MLA_OK); H >= 1 heads;
  *   block_size >= 1, num_blocks >= 0: cache geometry.
@@ -121,7 +121,9 @@ typedef enum mla_status {
  * (griddepcontrol.wait) only right before reading q_nope / q_pe; cache rows,
  * slot_mapping, positions, cos_sin and the scales are read without waiting
  * (PR #54896 report, 实现拆解 item 2).  CONTRACT: with this flag the previous
- * kernel may write q_nope and q_pe only.  The kernel signals its own
+ * kernel on `stream` may write q_nope and q_pe only, and must not read q_out
+ * or the cache rows this call writes (cache rows are written while that
+ * kernel may still be running).  The kernel signals its own
  * dependents (griddepcontrol.launch_dependents) only after all of its stores
  * (PR #54896 report, 评论区精华: the early trigger was a race and was moved
  * back to the end).
@@ -163,9 +165,12 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  * Tuning knobs of the plan (process-wide; not synchronised, set them before
  * launching from several threads).  The pages choose the small-batch split
  * for up to 64 tokens and note that the threshold may not suit other batch
- * sizes or hardware (PR #54896 report, 风险与影响 "risks" item 2); these let a
- * caller move it.  A value <= 0 keeps the current setting.
- *   split_max_tokens     T at or below which MLA_MODE_SPLIT is used (default 64)
+ * sizes or hardware (PR #54896 report, 风险与影响 "risks" item 2).  On B200
+ * the split kernel stays faster than the rows kernel up to about 4.6 K rows
+ * (T * (H + 1)) whatever H is (measured for H = 8, 16, 32, 128), so the
+ * default threshold counts rows, not tokens.  A value <= 0 keeps the current
+ * setting.
+ *   split_max_rows       T * (H + 1) at or below which MLA_MODE_SPLIT is used (default 4608)
  *   split_rows_per_block rows per block in MLA_MODE_SPLIT (block = 96 * this), at most 4
  *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
@@ -173,7 +178,7 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  * Larger values are clamped to those limits.
  */
 typedef struct mla_tuning {
-  int64_t split_max_tokens;
+  int64_t split_max_rows;
   int32_t split_rows_per_block;
   int32_t rows_warps_per_block;
   int32_t rows_blocks_per_sm;

@@ -47,16 +47,35 @@ MLA_API mla_status mla_harness_empty(int64_t blocks, int32_t threads, uint32_t f
 /*
  * Device check of the e4m3 quotient: for every fp32 bit pattern p in
  * [first, first + count) compares the epilogue's quotient x / scale with the
- * CUDA IEEE division __fdiv_rn (NaN equal to NaN) and the e4m3 bytes they
- * encode to.  result (device, 3 x uint64, overwritten): [0] inputs with
- * |x| >= 2^-100 and |x / scale| < 2^125 whose quotients differ (outside that
+ * CUDA IEEE division __fdiv_rn (NaN equal to NaN), and the e4m3 bytes the
+ * epilogue stores with those of the IEEE quotient, both for x as an fp32
+ * (the rotated pe values) and for the two halves of p as bf16 (the other
+ * values).  result (device, 3 x uint64, overwritten): [0] inputs with
+ * |x| >= 2^-100 and |x / scale| < 448 whose quotients differ (outside that
  * range the epilogue's quotient may differ in its last bits while its e4m3
- * byte, a signed zero below and +-448 above, may not), [1] inputs whose e4m3
- * bytes differ, [2] smallest pattern counted in [0] or [1] (UINT64_MAX if
- * none).  first + count <= 2^32.
+ * byte, a signed zero below and +-448 above, may not), [1] patterns whose
+ * e4m3 bytes differ on either path, [2] smallest pattern counted in [0] or
+ * [1] (UINT64_MAX if none).  first + count <= 2^32.
  */
 MLA_API mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t count,
                                  unsigned long long* result, mla_stream_t stream);
+
+/*
+ * Synthetic downstream consumer standing in for the attention kernel that
+ * reads the epilogue's outputs (PR #54896 report, 实现拆解 item 2: the
+ * epilogue's trigger lets the attention kernel overlap with it).  For every
+ * token t and head h it writes
+ *     scores[t * H + h] = sum_i dec(q_out[t, h, i]) * dec(cache.row(slot_mapping[t])[i])
+ * in fp32 (dec: bf16, or e4m3 with MLA_FLAG_Q_FP8 / MLA_FLAG_KV_FP8; the
+ * scales are not applied), or NaN when the slot is outside
+ * [0, cache_rows).  It reads slot_mapping before its griddepcontrol.wait
+ * and q_out and the cache only after it, so, launched with MLA_FLAG_PDL
+ * right behind the epilogue, it sees every store the epilogue made.
+ * q_out and cache: 16-byte aligned; scores: fp32 [T * H], 4-byte aligned.
+ */
+MLA_API mla_status mla_harness_consume(const void* q_out, const void* cache, const int64_t* slot_mapping,
+                                       int64_t T, int64_t H, int64_t cache_rows, uint32_t flags, float* scores,
+                                       mla_stream_t stream);
 
 #ifdef __cplusplus
 }

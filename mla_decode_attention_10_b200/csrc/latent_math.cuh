@@ -43,58 +43,123 @@ __device__ __forceinline__ void rope_pair(float a, float b, float c, float s, fl
   yb = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
 }
 
-// Per-tensor divisor.  `fast` holds when 2^-64 <= scale <= 2^64, where the
-// corrected-reciprocal quotient below is exact; otherwise quotients go
-// through the IEEE division intrinsic.
+// Per-tensor divisor.  `fast` holds when 2^-64 <= scale <= 2^64: there the
+// quotients come from the corrected reciprocal below; otherwise (zero,
+// negative, huge, tiny, NaN scales) from the IEEE division intrinsic.
 struct Divisor {
+  uint64_t s2;       // {s, s}
+  uint64_t ny2;      // {-RN(1/s), -RN(1/s)}
   float s;
-  float y;  // reciprocal of s, rounded to nearest
+  float nclamp;      // -B, B = smallest power of two >= 512 s
+  uint32_t nclamp2;  // -B as a bf16x2 pair (exact: B is a power of two)
   bool fast;
 };
+
+// {v, v} as one 64-bit operand of the packed f32x2 instructions.
+__device__ __forceinline__ uint64_t pair_of(float v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+  return r;
+}
 
 __device__ __forceinline__ Divisor make_divisor(float s) {
   Divisor d;
   d.s = s;
   d.fast = (s >= 0x1p-64f) && (s <= 0x1p64f);
-  d.y = d.fast ? __frcp_rn(s) : 1.0f;
+  d.s2 = pair_of(s);
+  d.ny2 = pair_of(d.fast ? -__frcp_rn(s) : -1.0f);
+  uint32_t b = __float_as_uint(d.fast ? 512.0f * s : 1.0f);
+  b = (b & 0x007fffffu) ? ((b & 0x7f800000u) + 0x00800000u) : b;
+  d.nclamp = -__uint_as_float(b);
+  const uint32_t hb = __float_as_uint(d.nclamp) >> 16;
+  d.nclamp2 = hb | (hb << 16);
   return d;
 }
 
-// x / s rounded to nearest even in fp32 (the IEEE quotient), for `fast` s.
+// -min(|x|, B) with the sign of x flipped; NaN stays NaN.  Values beyond B
+// divide to more than 512 and saturate to 448 in e4m3 whatever they are, so
+// the clamp changes no e4m3 result and keeps the quotient below 1024.
+__device__ __forceinline__ float neg_clamp(float x, const Divisor& d) {
+  float m;
+  asm("min.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(m) : "f"(x), "f"(d.nclamp));
+  return m;
+}
+
+// Same on a bf16x2 pair (both halves at once).
+__device__ __forceinline__ uint32_t neg_clamp_bf16x2(uint32_t w, const Divisor& d) {
+  uint32_t m;
+  asm("min.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(w), "r"(d.nclamp2));
+  return m;
+}
+
+// Quotients x / s of two values given as mx = -x (after neg_clamp), rounded
+// to nearest even in fp32, two lanes of fp32 arithmetic per instruction
+// (packed f32x2 multiply and fused multiply-add of sm_100).
 //
 // Method (Markstein, "Computation of elementary functions on the IBM RISC
 // System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also Cornea, Harrison
 // & Tang, "Scientific Computing on Itanium-based Systems", 2002): with
-// y = RN(1/s) and a quotient estimate q, the residual r = x - q s is exact in
-// one fused multiply-add whenever q is within an ulp of x/s, and
-// RN(q + r y) is then the correctly rounded quotient.  q0 = RN(x y) can be
-// up to ~1.5 ulp off, so one correction step first makes it faithful, and a
-// second one rounds it correctly.  Zero keeps the sign of x (s > 0).  When
-// |x y| is not below 2^126 (so that no correction step could overflow) or is
-// infinite or NaN, q0 is returned as is: the e4m3 result saturates to 448 or
-// is NaN whatever its last bits are.
-// Below |x| ~ 2^-102 the residual may underflow and the last bits of the
-// quotient may then differ from the IEEE quotient, but there |x / s| <= 2^-38,
-// which every e4m3 rounding sends to the same signed zero.
-__device__ __forceinline__ float div_rn(float x, const Divisor& d) {
-  if (!d.fast) return __fdiv_rn(x, d.s);
-  const float q0 = __fmul_rn(x, d.y);
-  const float r0 = __fmaf_rn(-q0, d.s, x);
-  const float q1 = __fmaf_rn(r0, d.y, q0);
-  const float r1 = __fmaf_rn(-q1, d.s, x);
-  const float q2 = __fmaf_rn(r1, d.y, q1);
-  return fabsf(q0) < 0x1p126f ? copysignf(q2, x) : q0;
+// y = RN(1/s) and a quotient estimate q within an ulp of x/s, the residual
+// r = x - q s is exact in one fused multiply-add and RN(q + r y) is the
+// correctly rounded quotient.  q0 = RN(x y) can be up to ~1.5 ulp off, so a
+// first correction makes it faithful and a second rounds it correctly.  The
+// steps are written on -x and -y so that every operand enters the FMA
+// unnegated: q0 = (-x)(-y), r = q s + (-x), q <- r (-y) + q; with these
+// forms a zero x gives a zero quotient of the same sign.  Below |x| ~ 2^-100
+// the residual may underflow and the last bits may differ from the IEEE
+// quotient, but there |x / s| <= 2^-36, which every e4m3 rounding sends to
+// the same signed zero.
+__device__ __forceinline__ void quotient_pair_neg(float mlo, float mhi, const Divisor& d, float& qlo,
+                                                  float& qhi) {
+  asm("{\n\t"
+      ".reg .b64 mx, q, r;\n\t"
+      "mov.b64 mx, {%2, %3};\n\t"
+      "mul.rn.f32x2 q, mx, %5;\n\t"
+      "fma.rn.f32x2 r, q, %4, mx;\n\t"
+      "fma.rn.f32x2 q, r, %5, q;\n\t"
+      "fma.rn.f32x2 r, q, %4, mx;\n\t"
+      "fma.rn.f32x2 q, r, %5, q;\n\t"
+      "mov.b64 {%0, %1}, q;\n\t"
+      "}"
+      : "=f"(qlo), "=f"(qhi)
+      : "f"(mlo), "f"(mhi), "l"(d.s2), "l"(d.ny2));
+}
+
+// e4m3 bytes of lo / s and hi / s for two fp32 values (lo in bits 0..7).
+// FAST: the divisor's scale is in [2^-64, 2^64] (d.fast), decided once per
+// kernel so that the per-element code has no branch.
+template <bool FAST>
+__device__ __forceinline__ uint32_t e4m3x2_of_f32(float lo, float hi, const Divisor& d) {
+  float qlo, qhi;
+  if (FAST) {
+    quotient_pair_neg(neg_clamp(lo, d), neg_clamp(hi, d), d, qlo, qhi);
+  } else {
+    qlo = __fdiv_rn(lo, d.s);
+    qhi = __fdiv_rn(hi, d.s);
+  }
+  return pack_e4m3x2(qlo, qhi);
+}
+
+// e4m3 bytes of the two bf16 of `w` divided by s (low half in bits 0..7).
+template <bool FAST>
+__device__ __forceinline__ uint32_t e4m3x2_of_bf16x2(uint32_t w, const Divisor& d) {
+  float qlo, qhi;
+  if (FAST) {
+    const uint32_t m = neg_clamp_bf16x2(w, d);
+    quotient_pair_neg(bf16_lo(m), bf16_hi(m), d, qlo, qhi);
+  } else {
+    qlo = __fdiv_rn(bf16_lo(w), d.s);
+    qhi = __fdiv_rn(bf16_hi(w), d.s);
+  }
+  return pack_e4m3x2(qlo, qhi);
 }
 
 // Eight bf16 (one 16-byte chunk) -> eight e4m3 bytes of x / s.
+template <bool FAST>
 __device__ __forceinline__ uint2 chunk_to_e4m3(const uint4 v, const Divisor& d) {
   uint2 o;
-  const uint32_t p0 = pack_e4m3x2(div_rn(bf16_lo(v.x), d), div_rn(bf16_hi(v.x), d));
-  const uint32_t p1 = pack_e4m3x2(div_rn(bf16_lo(v.y), d), div_rn(bf16_hi(v.y), d));
-  const uint32_t p2 = pack_e4m3x2(div_rn(bf16_lo(v.z), d), div_rn(bf16_hi(v.z), d));
-  const uint32_t p3 = pack_e4m3x2(div_rn(bf16_lo(v.w), d), div_rn(bf16_hi(v.w), d));
-  o.x = p0 | (p1 << 16);
-  o.y = p2 | (p3 << 16);
+  o.x = e4m3x2_of_bf16x2<FAST>(v.x, d) | (e4m3x2_of_bf16x2<FAST>(v.y, d) << 16);
+  o.y = e4m3x2_of_bf16x2<FAST>(v.z, d) | (e4m3x2_of_bf16x2<FAST>(v.w, d) << 16);
   return o;
 }
 

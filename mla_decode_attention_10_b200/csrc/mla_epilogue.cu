@@ -18,7 +18,9 @@
 //     dependent load (position -> table row) plus the data load.
 //   rows kernel (large T): one warp per row (lane: nope chunks lane and
 //     lane+32, pe pair lane); the grid is a multiple of the SM count sized to
-//     the resident blocks and strides over all rows.
+//     the resident blocks, each warp walks a contiguous range of rows, keeps
+//     the next row's loads in flight while it converts the current one, and
+//     looks up a token's rotation once for all of its adjacent rows.
 //
 // Row order: rows [0, T) are the T cache rows, rows [T, T + T*H) the query
 // rows in q_out order.  Cache rows never wait on the upstream kernel, so
@@ -43,7 +45,7 @@ constexpr int kHalfPe = 32;
 constexpr int kRow = 576;
 constexpr int kSplitThreadsPerRow = 96;
 constexpr int kSplitMaxRowsPerBlock = 4;  // 384 threads
-constexpr int kRowsMinBlocksPerSm = 5;    // register cap 48: five 256-thread blocks stay resident
+constexpr int kRowsMinBlocksPerSm = 5;    // register cap 64: four 256-thread blocks stay resident
 
 struct Args {
   const uint16_t* q_nope;
@@ -103,17 +105,17 @@ __device__ __forceinline__ Rot load_rotation(const Args& a, int64_t t, int i) {
 }
 
 // Nope chunk `chunk` (8 values) of a row: 16 bytes in, 16 (bf16) or 8 (e4m3) out.
-template <bool FP8>
+template <bool FP8, bool FAST>
 __device__ __forceinline__ void store_nope(uint8_t* dst, int chunk, const uint4 v, const Divisor& d) {
   if constexpr (FP8) {
-    *reinterpret_cast<uint2*>(dst + chunk * 8) = chunk_to_e4m3(v, d);
+    *reinterpret_cast<uint2*>(dst + chunk * 8) = chunk_to_e4m3<FAST>(v, d);
   } else {
     *reinterpret_cast<uint4*>(dst + chunk * 16) = v;
   }
 }
 
 // RoPE pair i of a row: pe[i] in the low half of `pe`, pe[i+32] in the high half.
-template <bool FP8, bool ROPE>
+template <bool FP8, bool ROPE, bool FAST>
 __device__ __forceinline__ void store_pe(uint8_t* dst, int i, uint32_t pe, const Rot& r, const Divisor& d) {
   float a = bf16_lo(pe);
   float b = bf16_hi(pe);
@@ -128,7 +130,7 @@ __device__ __forceinline__ void store_pe(uint8_t* dst, int i, uint32_t pe, const
     }
   }
   if constexpr (FP8) {
-    const uint32_t p = pack_e4m3x2(div_rn(a, d), div_rn(b, d));
+    const uint32_t p = e4m3x2_of_f32<FAST>(a, b, d);
     dst[kNope + i] = static_cast<uint8_t>(p & 0xffu);
     dst[kNope + kHalfPe + i] = static_cast<uint8_t>((p >> 8) & 0xffu);
   } else {
@@ -151,41 +153,37 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* pe, int i) {
 // split kernel: three warps per row
 // ------------------------------------------------------------------------------------
 
-template <bool FP8, bool ROPE>
-__device__ __forceinline__ void split_query_row(const Args& a, int64_t q, int part, int lane) {
+template <bool FP8, bool ROPE, bool FAST>
+__device__ __forceinline__ void split_query_row(const Args& a, int64_t q, int part, int lane, const Divisor& d) {
   const int64_t t = div_heads(a, q);
   const int64_t h = q - t * a.H;
   uint8_t* dst = a.q_out + q * (FP8 ? kRow : 2 * kRow);
-  Divisor d{};
-  if constexpr (FP8) d = make_divisor(__ldg(a.q_scale));
   if (part < 2) {
     const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh;
     const int chunk = part * 32 + lane;
     pdl_wait();
     const uint4 v = ld_chunk(src, chunk);
-    store_nope<FP8>(dst, chunk, v, d);
+    store_nope<FP8, FAST>(dst, chunk, v, d);
   } else {
     const uint16_t* src = a.q_pe + t * a.qp_st + h * a.qp_sh;
     Rot r{1.0f, 0.0f, false};
     if constexpr (ROPE) r = load_rotation(a, t, lane);
     pdl_wait();
     const uint32_t pe = ld_pair(src, lane);
-    store_pe<FP8, ROPE>(dst, lane, pe, r, d);
+    store_pe<FP8, ROPE, FAST>(dst, lane, pe, r, d);
   }
 }
 
-template <bool FP8, bool ROPE>
-__device__ __forceinline__ void split_cache_row(const Args& a, int64_t t, int part, int lane) {
+template <bool FP8, bool ROPE, bool FAST>
+__device__ __forceinline__ void split_cache_row(const Args& a, int64_t t, int part, int lane, const Divisor& d) {
   const int64_t slot = __ldg(a.slots + t);
   const bool in_range = slot >= 0 && slot < a.cache_rows;
   uint8_t* dst = a.cache + (in_range ? slot : 0) * (FP8 ? kRow : 2 * kRow);
-  Divisor d{};
-  if constexpr (FP8) d = make_divisor(__ldg(a.kv_scale));
   if (part < 2) {
     const int chunk = part * 32 + lane;
     const uint4 v = ld_chunk(a.kv_c + t * a.kv_st, chunk);
     if (part == 0 && lane == 0 && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
-    if (in_range) store_nope<FP8>(dst, chunk, v, d);
+    if (in_range) store_nope<FP8, FAST>(dst, chunk, v, d);
   } else {
     Rot r{1.0f, 0.0f, false};
     if constexpr (ROPE) {
@@ -193,7 +191,7 @@ __device__ __forceinline__ void split_cache_row(const Args& a, int64_t t, int pa
       if (lane == 0 && !r.on) report(a.status, MLA_STATUS_POS_RANGE);
     }
     const uint32_t pe = ld_pair(a.k_pe + t * a.kp_st, lane);
-    if (in_range) store_pe<FP8, ROPE>(dst, lane, pe, r, d);
+    if (in_range) store_pe<FP8, ROPE, FAST>(dst, lane, pe, r, d);
   }
 }
 
@@ -205,10 +203,26 @@ __global__ void __launch_bounds__(kSplitThreadsPerRow * kSplitMaxRowsPerBlock) m
   const int64_t g = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp / 3;
   const int part = warp % 3;
   if (g < a.rows) {
+    // the row's divisor (scales are read before any wait); quotients take the
+    // corrected-reciprocal path unless the scale is outside [2^-64, 2^64]
     if (g < a.T) {
-      split_cache_row<KVF8, ROPE>(a, g, part, lane);
+      Divisor d{};
+      d.fast = true;
+      if constexpr (KVF8) d = make_divisor(__ldg(a.kv_scale));
+      if (d.fast) {
+        split_cache_row<KVF8, ROPE, true>(a, g, part, lane, d);
+      } else {
+        split_cache_row<KVF8, ROPE, false>(a, g, part, lane, d);
+      }
     } else {
-      split_query_row<QF8, ROPE>(a, g - a.T, part, lane);
+      Divisor d{};
+      d.fast = true;
+      if constexpr (QF8) d = make_divisor(__ldg(a.q_scale));
+      if (d.fast) {
+        split_query_row<QF8, ROPE, true>(a, g - a.T, part, lane, d);
+      } else {
+        split_query_row<QF8, ROPE, false>(a, g - a.T, part, lane, d);
+      }
     }
   }
   pdl_trigger();
@@ -218,15 +232,11 @@ __global__ void __launch_bounds__(kSplitThreadsPerRow * kSplitMaxRowsPerBlock) m
 // rows kernel: one warp per row, grid-stride over rows
 // ------------------------------------------------------------------------------------
 
-template <bool QF8, bool KVF8, bool ROPE>
-__global__ void __launch_bounds__(256, kRowsMinBlocksPerSm) mla_epilogue_rows_kernel(const Args a) {
+template <bool QF8, bool KVF8, bool ROPE, bool FAST>
+__device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, const Divisor& dk) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-
-  Divisor dq{}, dk{};
-  if constexpr (QF8) dq = make_divisor(__ldg(a.q_scale));
-  if constexpr (KVF8) dk = make_divisor(__ldg(a.kv_scale));
   bool waited = false;
 
   for (int64_t g = wid; g < a.rows; g += warps) {
@@ -272,14 +282,29 @@ __global__ void __launch_bounds__(256, kRowsMinBlocksPerSm) mla_epilogue_rows_ke
     const uint32_t p = ld_pair(pe, lane);
     if (dst == nullptr) continue;
     if (is_cache) {
-      store_nope<KVF8>(dst, lane, n0, dk);
-      store_nope<KVF8>(dst, lane + 32, n1, dk);
-      store_pe<KVF8, ROPE>(dst, lane, p, rot, dk);
+      store_nope<KVF8, FAST>(dst, lane, n0, dk);
+      store_nope<KVF8, FAST>(dst, lane + 32, n1, dk);
+      store_pe<KVF8, ROPE, FAST>(dst, lane, p, rot, dk);
     } else {
-      store_nope<QF8>(dst, lane, n0, dq);
-      store_nope<QF8>(dst, lane + 32, n1, dq);
-      store_pe<QF8, ROPE>(dst, lane, p, rot, dq);
+      store_nope<QF8, FAST>(dst, lane, n0, dq);
+      store_nope<QF8, FAST>(dst, lane + 32, n1, dq);
+      store_pe<QF8, ROPE, FAST>(dst, lane, p, rot, dq);
     }
+  }
+}
+
+template <bool QF8, bool KVF8, bool ROPE>
+__global__ void __launch_bounds__(256, kRowsMinBlocksPerSm) mla_epilogue_rows_kernel(const Args a) {
+  // scales are read before any wait; the whole body takes the corrected-
+  // reciprocal quotient unless a scale is outside [2^-64, 2^64]
+  Divisor dq{}, dk{};
+  dq.fast = dk.fast = true;
+  if constexpr (QF8) dq = make_divisor(__ldg(a.q_scale));
+  if constexpr (KVF8) dk = make_divisor(__ldg(a.kv_scale));
+  if (dq.fast && dk.fast) {
+    rows_body<QF8, KVF8, ROPE, true>(a, dq, dk);
+  } else {
+    rows_body<QF8, KVF8, ROPE, false>(a, dq, dk);
   }
   pdl_trigger();
 }
@@ -315,7 +340,7 @@ constexpr uint32_t kKnownFlags = MLA_FLAG_ROPE | MLA_FLAG_Q_FP8 | MLA_FLAG_KV_FP
                                  MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS;
 constexpr int kMaxDevices = 64;
 
-mla_tuning g_tuning = {64, 2, 8, mla::kRowsMinBlocksPerSm};
+mla_tuning g_tuning = {4608, 2, 8, mla::kRowsMinBlocksPerSm};
 int g_sm_count[kMaxDevices] = {0};
 thread_local int32_t g_last_cuda_error = 0;
 
@@ -343,7 +368,7 @@ mla_status make_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla
   const int64_t rows = T * (H + 1);
   const bool split = (flags & MLA_FLAG_FORCE_SPLIT) ? true
                      : (flags & MLA_FLAG_FORCE_ROWS) ? false
-                                                      : (T <= g_tuning.split_max_tokens);
+                                                      : (rows <= g_tuning.split_max_rows);
   p->sm_count = sm_count;
   if (split) {
     const int32_t rpb = g_tuning.split_rows_per_block;
@@ -383,7 +408,7 @@ int32_t mla_last_cuda_error(void) { return g_last_cuda_error; }
 
 void mla_epilogue_set_tuning(const mla_tuning* t) {
   if (t == nullptr) return;
-  if (t->split_max_tokens > 0) g_tuning.split_max_tokens = t->split_max_tokens;
+  if (t->split_max_rows > 0) g_tuning.split_max_rows = t->split_max_rows;
   if (t->split_rows_per_block > 0)
     g_tuning.split_rows_per_block = t->split_rows_per_block < mla::kSplitMaxRowsPerBlock ? t->split_rows_per_block
                                                                                           : mla::kSplitMaxRowsPerBlock;

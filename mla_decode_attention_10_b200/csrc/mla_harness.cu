@@ -2,6 +2,7 @@
 // that sit beside the epilogue (declarations and contracts in mla_harness.h).
 
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "latent_math.cuh"
@@ -39,6 +40,15 @@ __global__ void __launch_bounds__(256) produce_kernel(const uint4* __restrict__ 
 
 __global__ void empty_kernel() {}
 
+// Quotient of one fp32 through the epilogue's e4m3 path (the pair function
+// with the second lane unused), returned as the fp32 quotient it encodes.
+__device__ __forceinline__ float epilogue_quotient(float x, const Divisor& d) {
+  if (!d.fast) return __fdiv_rn(x, d.s);
+  float q, unused;
+  quotient_pair_neg(neg_clamp(x, d), neg_clamp(0.0f, d), d, q, unused);
+  return q;
+}
+
 __global__ void __launch_bounds__(256) div_check_kernel(float scale, uint64_t first, uint64_t count,
                                                         unsigned long long* result) {
   const Divisor d = make_divisor(scale);
@@ -46,21 +56,26 @@ __global__ void __launch_bounds__(256) div_check_kernel(float scale, uint64_t fi
   unsigned long long bad_q = 0, bad_b = 0, lowest = ~0ull;
   for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
     const uint64_t p = first + i;
-    const float x = __uint_as_float(static_cast<uint32_t>(p));
-    const float q = div_rn(x, d);
+    const uint32_t w = static_cast<uint32_t>(p);
+    const float x = __uint_as_float(w);
+    const float q = epilogue_quotient(x, d);
     const float ref = __fdiv_rn(x, scale);
     const bool same_q = (__float_as_uint(q) == __float_as_uint(ref)) || (isnan(q) && isnan(ref));
-    const uint32_t bq = pack_e4m3x2(q, 0.0f) & 0xffu;
+    // fp32 path (rotated values): the byte the epilogue stores vs the byte of the IEEE quotient
+    const uint32_t bq = (d.fast ? e4m3x2_of_f32<true>(x, 0.0f, d) : e4m3x2_of_f32<false>(x, 0.0f, d)) & 0xffu;
     const uint32_t br = pack_e4m3x2(ref, 0.0f) & 0xffu;
-    // quotient bits are compared where div_rn computes the IEEE quotient:
-    // |x| >= 2^-100 (below, its residual may underflow; |x / scale| <= 2^-36
-    // rounds to a signed zero in e4m3) and |x / scale| < 2^125 (above, it
-    // returns the uncorrected product, which saturates in e4m3)
-    if (!same_q && fabsf(x) >= 0x1p-100f && !(fabsf(ref) >= 0x1p125f)) {
+    // bf16x2 path (unrotated inputs): the two halves of the pattern as bf16
+    const uint32_t bb = d.fast ? e4m3x2_of_bf16x2<true>(w, d) : e4m3x2_of_bf16x2<false>(w, d);
+    const uint32_t bbr = pack_e4m3x2(__fdiv_rn(bf16_lo(w), scale), __fdiv_rn(bf16_hi(w), scale));
+    // quotient bits are compared where they decide an e4m3 byte and the
+    // epilogue computes the IEEE quotient: |x| >= 2^-100 (below, the residual may
+    // underflow; |x / scale| <= 2^-36 rounds to a signed zero) and
+    // |x / scale| < 448 (above, the input is clamped; the byte saturates)
+    if (!same_q && fabsf(x) >= 0x1p-100f && !(fabsf(ref) >= 448.0f)) {
       ++bad_q;
       if (p < lowest) lowest = p;
     }
-    if (bq != br) {
+    if (bq != br || bb != bbr) {
       ++bad_b;
       if (p < lowest) lowest = p;
     }
@@ -68,6 +83,43 @@ __global__ void __launch_bounds__(256) div_check_kernel(float scale, uint64_t fi
   if (bad_q) atomicAdd(result + 0, bad_q);
   if (bad_b) atomicAdd(result + 1, bad_b);
   if (lowest != ~0ull) atomicMin(result + 2, lowest);
+}
+
+// e4m3 byte -> fp32 (exact: every e4m3 value is an fp16 value).
+__device__ __forceinline__ float e4m3_to_f32(uint8_t b) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(b)));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xffffu)));
+}
+
+template <bool QF8, bool KVF8>
+__global__ void __launch_bounds__(256) consume_kernel(const uint8_t* q_out, const uint8_t* cache,
+                                                      const int64_t* slots, int64_t T, int64_t H,
+                                                      int64_t cache_rows, float* scores) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  // slot_mapping is not written by the epilogue: read it before waiting
+  int64_t slot = first < T * H ? __ldg(slots + first / H) : 0;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int64_t r = first; r < T * H; r += warps) {
+    if (r != first) slot = __ldg(slots + r / H);
+    if (slot < 0 || slot >= cache_rows) {
+      if (lane == 0) scores[r] = __int_as_float(0x7fc00000);
+      continue;
+    }
+    const uint8_t* q = q_out + r * (QF8 ? 576 : 1152);
+    const uint8_t* k = cache + slot * (KVF8 ? 576 : 1152);
+    float acc = 0.0f;
+    for (int i = lane; i < 576; i += 32) {
+      const float qv = QF8 ? e4m3_to_f32(__ldcg(q + i)) : bf16_bits(__ldcg(reinterpret_cast<const uint16_t*>(q) + i));
+      const float kv = KVF8 ? e4m3_to_f32(__ldcg(k + i)) : bf16_bits(__ldcg(reinterpret_cast<const uint16_t*>(k) + i));
+      acc = __fmaf_rn(qv, kv, acc);
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) scores[r] = acc;
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -149,6 +201,31 @@ mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t count, un
   if (count == 0) return MLA_OK;
   void* args[] = {&scale, &first, &count, &result};
   return launch(reinterpret_cast<const void*>(&div_check_kernel), dim3(148 * 16), dim3(256), false, s, args);
+}
+
+mla_status mla_harness_consume(const void* q_out, const void* cache, const int64_t* slot_mapping, int64_t T,
+                               int64_t H, int64_t cache_rows, uint32_t flags, float* scores, mla_stream_t stream) {
+  using namespace mla::harness;
+  if ((flags & ~(MLA_FLAG_Q_FP8 | MLA_FLAG_KV_FP8 | MLA_FLAG_PDL)) != 0) return MLA_ERR_UNSUPPORTED;
+  if (T < 0 || H < 1 || cache_rows < 0 || T > (INT64_C(1) << 31) / H) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!q_out || !slot_mapping || !scores || (!cache && cache_rows > 0)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_out) || (cache && !aligned16(cache)) || (reinterpret_cast<uintptr_t>(scores) & 3u) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return MLA_ERR_ALIGNMENT;
+  const int64_t rows = T * H;
+  int64_t blocks = (rows + 7) / 8;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  const bool qf8 = (flags & MLA_FLAG_Q_FP8) != 0, kvf8 = (flags & MLA_FLAG_KV_FP8) != 0;
+  const void* fn = qf8 ? (kvf8 ? reinterpret_cast<const void*>(&consume_kernel<true, true>)
+                               : reinterpret_cast<const void*>(&consume_kernel<true, false>))
+                       : (kvf8 ? reinterpret_cast<const void*>(&consume_kernel<false, true>)
+                               : reinterpret_cast<const void*>(&consume_kernel<false, false>));
+  const uint8_t* q = static_cast<const uint8_t*>(q_out);
+  const uint8_t* c = static_cast<const uint8_t*>(cache);
+  void* args[] = {&q, &c, &slot_mapping, &T, &H, &cache_rows, &scores};
+  return launch(fn, dim3(static_cast<unsigned>(blocks)), dim3(256), (flags & MLA_FLAG_PDL) != 0,
+                reinterpret_cast<cudaStream_t>(stream), args);
 }
 
 }  // extern "C"

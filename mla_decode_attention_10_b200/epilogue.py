@@ -57,7 +57,7 @@ class mla_plan(ctypes.Structure):
 
 
 class mla_tuning(ctypes.Structure):
-    _fields_ = [("split_max_tokens", ctypes.c_int64), ("split_rows_per_block", ctypes.c_int32),
+    _fields_ = [("split_max_rows", ctypes.c_int64), ("split_rows_per_block", ctypes.c_int32),
                 ("rows_warps_per_block", ctypes.c_int32), ("rows_blocks_per_sm", ctypes.c_int32)]
 
 
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.mla_harness_produce.argtypes = [vp, vp, vp, i64, i64, vp, i64, i64, i64, i64, u32, vp]
         L.mla_harness_empty.restype = ctypes.c_int
         L.mla_harness_empty.argtypes = [i64, i32, u32, vp]
+        L.mla_harness_consume.restype = ctypes.c_int
+        L.mla_harness_consume.argtypes = [vp, vp, vp, i64, i64, i64, u32, vp, vp]
         L.mla_harness_div_check.restype = ctypes.c_int
         L.mla_harness_div_check.argtypes = [ctypes.c_float, u64, u64, vp, vp]
         _lib = L
@@ -118,9 +120,9 @@ def mla_epilogue_plan(T: int, H: int, flags: int = 0, sm_count: int = 0) -> mla_
     return p
 
 
-def mla_epilogue_set_tuning(split_max_tokens: int = 0, split_rows_per_block: int = 0,
+def mla_epilogue_set_tuning(split_max_rows: int = 0, split_rows_per_block: int = 0,
                             rows_warps_per_block: int = 0, rows_blocks_per_sm: int = 0) -> None:
-    t = mla_tuning(split_max_tokens, split_rows_per_block, rows_warps_per_block, rows_blocks_per_sm)
+    t = mla_tuning(split_max_rows, split_rows_per_block, rows_warps_per_block, rows_blocks_per_sm)
     lib().mla_epilogue_set_tuning(ctypes.byref(t))
 
 
@@ -146,6 +148,10 @@ def mla_harness_produce(src_nope, src_pe, q_nope, q_nope_stride_t, q_nope_stride
 
 def mla_harness_empty(blocks: int, threads: int, flags: int, stream) -> int:
     return lib().mla_harness_empty(blocks, threads, flags, stream)
+
+
+def mla_harness_consume(q_out, cache, slot_mapping, T, H, cache_rows, flags, scores, stream) -> int:
+    return lib().mla_harness_consume(q_out, cache, slot_mapping, T, H, cache_rows, flags, scores, stream)
 
 
 def mla_harness_div_check(scale: float, first: int, count: int, result, stream) -> int:

@@ -136,13 +136,20 @@ def test_plan_modes_and_grids(lib):
     p = E.mla_epilogue_plan(64, 16, 0, sm_count=148)
     assert p.mode == E.MLA_MODE_SPLIT and p.threads_per_block == 96 * p.rows_per_block
     assert p.blocks == -(-64 * 17 // p.rows_per_block)
-    p = E.mla_epilogue_plan(65, 16, 0, sm_count=148)
+    # the default split threshold counts rows: 4608 = 271 tokens x 17 rows, rounded up
+    assert E.mla_epilogue_get_tuning().split_max_rows == 4608
+    assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
+    assert E.mla_epilogue_plan(271, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
+    assert E.mla_epilogue_plan(272, 16, 0, sm_count=148).mode == E.MLA_MODE_ROWS
+    assert E.mla_epilogue_plan(32, 128, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
+    assert E.mla_epilogue_plan(36, 128, 0, sm_count=148).mode == E.MLA_MODE_ROWS
+    p = E.mla_epilogue_plan(300, 16, 0, sm_count=148)
     assert p.mode == E.MLA_MODE_ROWS and p.threads_per_block % 32 == 0
     assert p.blocks <= 148 * E.mla_epilogue_get_tuning().rows_blocks_per_sm
-    assert p.blocks % 148 == 0 or p.blocks * (p.threads_per_block // 32) >= 65 * 17
     assert E.mla_epilogue_plan(1, 16, E.MLA_FLAG_FORCE_ROWS, sm_count=148).mode == E.MLA_MODE_ROWS
     assert E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148).mode == E.MLA_MODE_SPLIT
     big = E.mla_epilogue_plan(8192, 16, 0, sm_count=148)
+    assert big.mode == E.MLA_MODE_ROWS
     assert big.blocks == 148 * E.mla_epilogue_get_tuning().rows_blocks_per_sm
     with pytest.raises(E.MlaError):
         E.mla_epilogue_plan(0, 16, 0, sm_count=148)
@@ -153,15 +160,16 @@ def test_plan_modes_and_grids(lib):
 def test_tuning_moves_the_threshold_and_clamps(lib):
     old = E.mla_epilogue_get_tuning()
     try:
-        E.mla_epilogue_set_tuning(split_max_tokens=128)
-        assert E.mla_epilogue_plan(100, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
+        E.mla_epilogue_set_tuning(split_max_rows=64 * 17)
+        assert E.mla_epilogue_plan(64, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
+        assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_ROWS
         E.mla_epilogue_set_tuning(split_rows_per_block=99, rows_warps_per_block=99, rows_blocks_per_sm=99)
         t = E.mla_epilogue_get_tuning()
         assert t.split_rows_per_block == 4 and t.rows_warps_per_block == 8 and t.rows_blocks_per_sm <= 5
         E.mla_epilogue_set_tuning()  # all zero: unchanged
-        assert E.mla_epilogue_get_tuning().split_max_tokens == 128
+        assert E.mla_epilogue_get_tuning().split_max_rows == 64 * 17
     finally:
-        E.mla_epilogue_set_tuning(old.split_max_tokens, old.split_rows_per_block,
+        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_rows_per_block,
                                   old.rows_warps_per_block, old.rows_blocks_per_sm)
 
 
@@ -187,3 +195,8 @@ def test_harness_validation(lib, kw, code):
     assert E.mla_harness_empty(1, 2048, 0, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_div_check(1.0, 0, 2 ** 32 + 1, A, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_div_check(1.0, 0, 1, None, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_consume(A, A, A, 4, 16, 64, 64, A, None) == E.MLA_ERR_UNSUPPORTED
+    assert E.mla_harness_consume(A, A, A, -1, 16, 64, 0, A, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_consume(None, A, A, 4, 16, 64, 0, A, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_consume(A + 8, A, A, 4, 16, 64, 0, A, None) == E.MLA_ERR_ALIGNMENT
+    assert E.mla_harness_consume(A, A, A, 0, 16, 64, 0, None, None) == E.MLA_OK

@@ -110,8 +110,9 @@ DIV_SCALES = [0.05, 1.0, 0.37, 3.0, 7.0, 0.9, 1.0 / 3.0, 2.0 ** -64, 2.0 ** 64, 
 @pytest.mark.parametrize("scale", DIV_SCALES)
 def test_quotient_equals_ieee_division_for_every_fp32(scale):
     """The epilogue's x / scale against CUDA's IEEE division for all 2^32 fp32
-    bit patterns: the same e4m3 byte everywhere, and the same quotient bits
-    for 2^-100 <= |x| and |x / scale| < 2^125 (NaN counted equal)."""
+    bit patterns: the same e4m3 byte everywhere (as fp32, and each half as
+    bf16), and the same quotient bits for 2^-100 <= |x| and |x / scale| < 448
+    (NaN counted equal)."""
     res = torch.zeros(3, dtype=torch.int64, device="cuda")
     rc = E.mla_harness_div_check(scale, 0, 2 ** 32, res.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert rc == E.MLA_OK
@@ -210,3 +211,21 @@ def test_torch_convenience_wrapper_matches_oracle():
                                                     d.slot_mapping, positions=d.positions,
                                                     cos_sin=d.cos_sin, kv_scale=d.kv_scale,
                                                     extra_flags=E.MLA_FLAG_FORCE_ROWS | E.MLA_FLAG_FORCE_SPLIT)
+
+
+@pytest.mark.parametrize("scale", [1e-25, 5e25, -0.5, 2.0 ** -70, 0.0, float("inf")])
+@pytest.mark.parametrize("force", FORCE[1:])
+def test_scales_outside_the_fast_range(scale, force):
+    """Scales outside [2^-64, 2^64] (and zero, negative, infinite ones) take
+    the IEEE-division path in both kernels: bytes equal the oracle's, NaN
+    results compared as NaN (the sign of a NaN code is not specified)."""
+    w = W.make("scales", 9, 16, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8, seed=12, num_blocks=1,
+               block_size=16, std=3.0, rope_rows=64, cache_fill="random")
+    w.q_scale.fill_(scale)
+    w.kv_scale.fill_(scale)
+    qg, cg, _ = run_gpu(w, extra_flags=force)
+    qo, co, _ = run_oracle(w)
+    for g, o, what in ((qg, qo, "q_out"), (cg, co, "cache")):
+        nan = (o & 0x7F) == 0x7F
+        assert torch.all((g[nan] & 0x7F) == 0x7F), what
+        assert torch.equal(g[~nan], o[~nan]), what
