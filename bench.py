@@ -46,6 +46,20 @@ METRIC = "µs/call and achieved HBM GB/s (fraction of ~8 TB/s) vs T for MLA epil
 UNIT = "µs/call"
 HEADLINE = "split_boundary_t64_h16_rope"
 FALLBACK_HBM_GBS = 6650.0
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the epilogue kernel, from ncu captures of `bench.py --steps 3 --warmup 3
+# --no-sweep --no-cpu-baseline --workload <name>` (third launch; summaries in
+# profiles/).  Keyed by a hash of the kernel sources they were taken on: a
+# changed kernel reports null until it is captured again.
+KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
+                  "mla_decode_attention_10_b200/csrc/latent_math.cuh", "include/mla_epilogue.h")
+TRAFFIC_SOURCE_HASH = "097d8a46e6e610e8"
+TRAFFIC_BYTES = {
+    "split_boundary_t64_h16_rope": 1277952 + 0,
+    "prefill_t1024_h128_strided": 152627456 + 102022400,
+    "batch_t8192_h16_pdl_fp8": 164003328 + 55213568,
+}
 L2_BYTES = 126 * 2 ** 20
 GRAPH_CALLS = 500
 
@@ -206,6 +220,22 @@ def timed(runner: GraphRunner, device, flush: bool = True) -> float:
     torch.cuda.synchronize()
     barrier(device)
     return max_over_ranks(e0.elapsed_time(e1), device)
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(name: str):
+    """Captured DRAM bytes per launch for `name`, or None (not captured, or the kernel changed since)."""
+    if name not in TRAFFIC_BYTES or kernel_source_hash() != TRAFFIC_SOURCE_HASH:
+        return None
+    return TRAFFIC_BYTES[name]
 
 
 def measured_hbm_gbs():
@@ -418,10 +448,12 @@ def run_ours(args, rank, world, local_rank):
                             "headline reads HBM)"},
         "producer_epilogue_consumer": chain,
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(gbs / peak, 4), "traffic": None,
+                     "frac": round(gbs / peak, 4), "traffic": traffic_for(args.workload),
+                     "algorithmic_bytes": w0.algorithmic_bytes(),
                      "peak_source": peak_note,
                      "note": "decode-size call: launch and memory latency bound, not bandwidth bound; "
-                             "see sweep for the bandwidth-bound sizes"},
+                             "see sweep for the bandwidth-bound sizes. traffic counts DRAM bytes inside the "
+                             "launch: written rows stay in L2 (write-back) and reach DRAM later"},
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clocks,
@@ -458,7 +490,7 @@ def sweep_one(name, E, stream, device, peak, epilogue_step, floor_step, measure,
     gbs = w0.algorithmic_bytes() / (us * 1e-6) / 1e9
     out = {"workload": name, "T": w0.T, "H": w0.H, "flags": flag_names(w0.flags),
            "mode": "split" if plan.mode == E.MLA_MODE_SPLIT else "rows",
-           "bytes_per_call": w0.algorithmic_bytes(), "us_per_call": round(us, 3),
+           "bytes_per_call": w0.algorithmic_bytes(), "traffic": traffic_for(name), "us_per_call": round(us, 3),
            "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "launch_floor_us": round(floor_us, 3),
            "floor_ratio": round(us / floor_us, 3), "calls": n, "sets": len(ds.sets),
            "l2": f"{ds.touched / 2 ** 20:.0f} MiB touched per rotation"}
@@ -513,10 +545,18 @@ def producer_consumer_chain(ds, E, stream, device, n, warmup):
     scores = torch.empty(w0.T * w0.H, dtype=torch.float32, device=device)
     cflags = (E.MLA_FLAG_Q_FP8 if w0.q_fp8 else 0) | (E.MLA_FLAG_KV_FP8 if w0.kv_fp8 else 0)
 
+    sources = {}
+
+    def source(k):
+        # the producer reads contiguous [T,H,512] / [T,H,64] buffers
+        if k not in sources:
+            d, _, src = ds.sets[k]
+            sources[k] = src if src is not None else (d.q_nope.contiguous(), d.q_pe.contiguous())
+        return sources[k]
+
     def prod(i):
-        d, _, src = ds.sets[i % S]
-        sn, sp = src if src is not None else (ds.sets[(i + 1) % S][0].q_nope, ds.sets[(i + 1) % S][0].q_pe)
-        assert sn.is_contiguous() and sp.is_contiguous()
+        d, _, _ = ds.sets[i % S]
+        sn, sp = source((i + 1) % S) if ds.sets[i % S][2] is None else source(i % S)
         rc = E.mla_harness_produce(sn.data_ptr(), sp.data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0),
                                    d.q_nope.stride(1), d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1),
                                    d.T, d.H, 0, stream.cuda_stream)

@@ -174,7 +174,8 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  *   split_rows_per_block rows per block in MLA_MODE_SPLIT (block = 96 * this), at most 4
  *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
- *                        the 5 that the kernel's register cap keeps resident
+ *                        the number the kernel's register cap keeps resident
+ *                        (6 with an e4m3 output, 5 without)
  * Larger values are clamped to those limits.
  */
 typedef struct mla_tuning {

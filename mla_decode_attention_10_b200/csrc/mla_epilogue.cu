@@ -45,7 +45,13 @@ constexpr int kHalfPe = 32;
 constexpr int kRow = 576;
 constexpr int kSplitThreadsPerRow = 96;
 constexpr int kSplitMaxRowsPerBlock = 4;  // 384 threads
-constexpr int kRowsMinBlocksPerSm = 5;    // register cap 64: four 256-thread blocks stay resident
+// Resident 256-thread blocks per SM the rows kernel is compiled for: 5 (a
+// 48-register cap) for bf16 outputs; 6 (40 registers) when an output is
+// e4m3, whose arithmetic leaves the kernel short of memory parallelism at 5
+// (measured on B200: 0.75 -> 0.78 of copy bandwidth for T=8192, H=16; the
+// bf16 variants lose at 6).
+constexpr int kRowsMaxBlocksPerSm = 6;
+constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 6 : 5; }
 
 struct Args {
   const uint16_t* q_nope;
@@ -294,7 +300,7 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
 }
 
 template <bool QF8, bool KVF8, bool ROPE>
-__global__ void __launch_bounds__(256, kRowsMinBlocksPerSm) mla_epilogue_rows_kernel(const Args a) {
+__global__ void __launch_bounds__(256, rows_blocks_per_sm(QF8, KVF8)) mla_epilogue_rows_kernel(const Args a) {
   // scales are read before any wait; the whole body takes the corrected-
   // reciprocal quotient unless a scale is outside [2^-64, 2^64]
   Divisor dq{}, dk{};
@@ -340,7 +346,7 @@ constexpr uint32_t kKnownFlags = MLA_FLAG_ROPE | MLA_FLAG_Q_FP8 | MLA_FLAG_KV_FP
                                  MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS;
 constexpr int kMaxDevices = 64;
 
-mla_tuning g_tuning = {4608, 2, 8, mla::kRowsMinBlocksPerSm};
+mla_tuning g_tuning = {4608, 2, 8, mla::kRowsMaxBlocksPerSm};
 int g_sm_count[kMaxDevices] = {0};
 thread_local int32_t g_last_cuda_error = 0;
 
@@ -380,7 +386,9 @@ mla_status make_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla
     const int32_t w = g_tuning.rows_warps_per_block;
     const int64_t per_block = w;
     const int64_t need = (rows + per_block - 1) / per_block;
-    const int64_t cap = static_cast<int64_t>(sm_count) * g_tuning.rows_blocks_per_sm;
+    const int32_t resident = mla::rows_blocks_per_sm((flags & MLA_FLAG_Q_FP8) != 0, (flags & MLA_FLAG_KV_FP8) != 0);
+    const int32_t per_sm = g_tuning.rows_blocks_per_sm < resident ? g_tuning.rows_blocks_per_sm : resident;
+    const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
     p->mode = MLA_MODE_ROWS;
     p->rows_per_block = 1;
     p->threads_per_block = 32 * w;
@@ -415,7 +423,7 @@ void mla_epilogue_set_tuning(const mla_tuning* t) {
   if (t->rows_warps_per_block > 0) g_tuning.rows_warps_per_block = t->rows_warps_per_block < 8 ? t->rows_warps_per_block : 8;
   if (t->rows_blocks_per_sm > 0)
     g_tuning.rows_blocks_per_sm =
-        t->rows_blocks_per_sm < mla::kRowsMinBlocksPerSm ? t->rows_blocks_per_sm : mla::kRowsMinBlocksPerSm;
+        t->rows_blocks_per_sm < mla::kRowsMaxBlocksPerSm ? t->rows_blocks_per_sm : mla::kRowsMaxBlocksPerSm;
 }
 
 void mla_epilogue_get_tuning(mla_tuning* out) {

@@ -149,8 +149,9 @@ def test_plan_modes_and_grids(lib):
     assert E.mla_epilogue_plan(1, 16, E.MLA_FLAG_FORCE_ROWS, sm_count=148).mode == E.MLA_MODE_ROWS
     assert E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148).mode == E.MLA_MODE_SPLIT
     big = E.mla_epilogue_plan(8192, 16, 0, sm_count=148)
-    assert big.mode == E.MLA_MODE_ROWS
-    assert big.blocks == 148 * E.mla_epilogue_get_tuning().rows_blocks_per_sm
+    assert big.mode == E.MLA_MODE_ROWS and big.blocks == 148 * 5
+    big8 = E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_Q_FP8 | E.MLA_FLAG_KV_FP8, sm_count=148)
+    assert big8.mode == E.MLA_MODE_ROWS and big8.blocks == 148 * 6
     with pytest.raises(E.MlaError):
         E.mla_epilogue_plan(0, 16, 0, sm_count=148)
     with pytest.raises(E.MlaError):
@@ -165,7 +166,7 @@ def test_tuning_moves_the_threshold_and_clamps(lib):
         assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_ROWS
         E.mla_epilogue_set_tuning(split_rows_per_block=99, rows_warps_per_block=99, rows_blocks_per_sm=99)
         t = E.mla_epilogue_get_tuning()
-        assert t.split_rows_per_block == 4 and t.rows_warps_per_block == 8 and t.rows_blocks_per_sm <= 5
+        assert t.split_rows_per_block == 4 and t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 6
         E.mla_epilogue_set_tuning()  # all zero: unchanged
         assert E.mla_epilogue_get_tuning().split_max_rows == 64 * 17
     finally:
