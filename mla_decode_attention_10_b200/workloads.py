@@ -254,3 +254,84 @@ def all_named() -> Dict[str, "callable"]:
 
 def names() -> List[str]:
     return list(RECIPES.keys())
+
+
+# --- the query side with the absorption product folded in ----------------------------
+
+ABSORB_IN = 128  # nope head dim before absorption
+
+
+@dataclasses.dataclass
+class AbsorbWorkload:
+    """Inputs of the absorbed-query rows: q_out[t,h] = enc([q_nope_c[t,h] @ W_UK[h]^T | rope(q_pe[t,h])])."""
+
+    name: str
+    T: int
+    H: int
+    flags: int
+    q_nope_c: torch.Tensor          # bf16 [T, H, 128], inner stride 1 (may be a view)
+    w_uk: torch.Tensor              # bf16 [H, 512, 128] contiguous (per head: 512 latent rows of 128)
+    q_pe: torch.Tensor              # bf16 [T, H, 64]
+    positions: Optional[torch.Tensor] = None
+    cos_sin: Optional[torch.Tensor] = None
+    q_scale: Optional[torch.Tensor] = None
+    recipe: str = ""
+
+    @property
+    def q_fp8(self) -> bool:
+        return bool(self.flags & FLAG_Q_FP8)
+
+    def q_out_dtype(self) -> torch.dtype:
+        return torch.uint8 if self.q_fp8 else torch.bfloat16
+
+    def to(self, device) -> "AbsorbWorkload":
+        out = {}
+        for f in dataclasses.fields(self):
+            v = getattr(self, f.name)
+            out[f.name] = _move(v, device) if isinstance(v, torch.Tensor) else v
+        return AbsorbWorkload(**out)
+
+    def flops(self) -> int:
+        return 2 * self.T * self.H * ABSORB_IN * NOPE
+
+    def algorithmic_bytes(self) -> int:
+        """Every input read once (the weights once per call), every output row written once."""
+        T, H = self.T, self.H
+        rd = T * H * ABSORB_IN * 2 + H * NOPE * ABSORB_IN * 2 + T * H * PE * 2
+        if self.flags & FLAG_ROPE:
+            rd += T * (4 + PE * 4)
+        if self.q_fp8:
+            rd += 4
+        return rd + T * H * ROW * (1 if self.q_fp8 else 2)
+
+
+def make_absorb(name: str, T: int, H: int, flags: int, *, seed: int, std: float = 1.0,
+                rope_rows: int = 32768, scale: float = 0.05, q_nope_row: int = ABSORB_IN,
+                recipe: str = "") -> AbsorbWorkload:
+    """Seeded absorbed-query inputs.  Draw order: q_nope_c ~ N(0, std), W_UK ~
+    N(0, 1/128) (so the 128-term products are O(std)), q_pe ~ N(0, std), then
+    positions uniform in [0, rope_rows).  ``q_nope_row`` > 128 makes q_nope_c
+    a view into a wider row-major buffer."""
+    g = torch.Generator().manual_seed(seed)
+    qc = _randn_bf16(g, (T, H, q_nope_row), std)[:, :, :ABSORB_IN]
+    w = _randn_bf16(g, (H, NOPE, ABSORB_IN), 1.0 / (ABSORB_IN ** 0.5))
+    qp = _randn_bf16(g, (T, H, PE), std)
+    positions = cos_sin = None
+    if flags & FLAG_ROPE:
+        positions = torch.randint(0, rope_rows, (T,), generator=g, dtype=torch.int64).to(torch.int32)
+        cos_sin = rope_table(rope_rows)
+    q_scale = torch.tensor([scale], dtype=torch.float32) if flags & FLAG_Q_FP8 else None
+    return AbsorbWorkload(name=name, T=T, H=H, flags=flags, q_nope_c=qc, w_uk=w, q_pe=qp, positions=positions,
+                          cos_sin=cos_sin, q_scale=q_scale, recipe=recipe)
+
+
+def absorb_t8192_h16_fp8() -> AbsorbWorkload:
+    return make_absorb("absorb_t8192_h16_rope_fp8", 8192, 16, FLAG_ROPE | FLAG_Q_FP8, seed=0, rope_rows=131072,
+                       recipe="T=8192 H=16: q_nope_c [8192,16,128] and q_pe bf16 N(0,1), W_UK [16,512,128] "
+                              "N(0,1/128), RoPE (131072-row table), e4m3 scale 0.05, seed 0")
+
+
+def absorb_t64_h16() -> AbsorbWorkload:
+    return make_absorb("absorb_t64_h16_rope", 64, 16, FLAG_ROPE, seed=3,
+                       recipe="T=64 H=16: q_nope_c [64,16,128] and q_pe bf16 N(0,1), W_UK [16,512,128] N(0,1/128), "
+                              "RoPE (32768-row table), bf16 out, seed 3")

@@ -40,6 +40,9 @@ def lib() -> ctypes.CDLL:
         L.mla_oracle_run.argtypes = [vp, i64, i64, vp, i64, i64, vp, i64, vp, i64,
                                      vp, vp, vp, i64, vp, vp,
                                      i64, i64, i64, i64, u32, vp, vp, vp]
+        L.mla_oracle_absorb_run.restype = ctypes.c_int
+        L.mla_oracle_absorb_run.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, vp,
+                                            i64, i64, u32, vp, vp]
         L.mla_oracle_bf16_to_f32.restype = ctypes.c_float
         L.mla_oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
         L.mla_oracle_f32_to_bf16.restype = ctypes.c_uint16
@@ -96,6 +99,29 @@ def run(q_nope: torch.Tensor, q_pe: torch.Tensor, kv_c: torch.Tensor, k_pe: torc
         _ptr(q_scale), _ptr(kv_scale),
         T, H, cache.shape[1], cache.shape[0], flags,
         _ptr(q_out), _ptr(cache), ctypes.addressof(status))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return q_out, status.value
+
+
+def absorb_run(q_nope_c: torch.Tensor, w_uk: torch.Tensor, q_pe: torch.Tensor, flags: int,
+               positions: Optional[torch.Tensor] = None, cos_sin: Optional[torch.Tensor] = None,
+               q_scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, int]:
+    """Latent query rows from the absorption product (see mla_oracle_absorb_run):
+    q_nope_c [T,H,128] bf16, w_uk [H,512,128] bf16 contiguous, q_pe [T,H,64] bf16.
+    Returns (q_out [T,H,576] bf16 or uint8 e4m3, status)."""
+    T, H = q_nope_c.shape[0], q_nope_c.shape[1]
+    assert q_nope_c.dtype == torch.bfloat16 and q_nope_c.stride(-1) == 1 and q_nope_c.shape[2] == 128
+    assert w_uk.dtype == torch.bfloat16 and w_uk.is_contiguous() and tuple(w_uk.shape) == (H, 512, 128)
+    assert q_pe.dtype == torch.bfloat16 and q_pe.stride(-1) == 1
+    q_fp8 = bool(flags & FLAG_Q_FP8)
+    q_out = torch.empty((T, H, ROW), dtype=torch.uint8 if q_fp8 else torch.bfloat16)
+    status = ctypes.c_int32(0)
+    rc = lib().mla_oracle_absorb_run(
+        _ptr(q_nope_c), q_nope_c.stride(0), q_nope_c.stride(1), _ptr(w_uk),
+        _ptr(q_pe), q_pe.stride(0), q_pe.stride(1),
+        _ptr(positions), _ptr(cos_sin), cos_sin.shape[0] if cos_sin is not None else 0,
+        _ptr(q_scale), T, H, flags, _ptr(q_out), ctypes.addressof(status))
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return q_out, status.value

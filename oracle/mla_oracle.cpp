@@ -123,12 +123,12 @@ uint8_t f32_to_e4m3_satfinite(float f) {
   return static_cast<uint8_t>(sign | static_cast<uint8_t>((e + 7) << 3) | static_cast<uint8_t>(k));
 }
 
-// One latent row: 576 fp32 values from bf16 sources, optionally rotated,
-// then encoded to bf16 or to e4m3.
-void build_latent_row(const uint16_t* nope, const uint16_t* pe, const float* rope_row,
-                      bool fp8, float scale, uint8_t* dst) {
+// One latent row from 512 fp32 nope values and 64 bf16 pe values: the pe
+// part optionally rotated, then all 576 encoded to bf16 or to e4m3.
+void encode_latent_row(const float* nope, const uint16_t* pe, const float* rope_row,
+                       bool fp8, float scale, uint8_t* dst) {
   float x[kRow];
-  for (int i = 0; i < kNope; ++i) x[i] = bf16_to_f32(nope[i]);
+  for (int i = 0; i < kNope; ++i) x[i] = nope[i];
   for (int i = 0; i < kPe; ++i) x[kNope + i] = bf16_to_f32(pe[i]);
 
   float y[kRow];
@@ -160,6 +160,14 @@ void build_latent_row(const uint16_t* nope, const uint16_t* pe, const float* rop
       std::memcpy(dst + 2 * i, &h, sizeof h);
     }
   }
+}
+
+// One latent row from bf16 sources (the epilogue's rows).
+void build_latent_row(const uint16_t* nope, const uint16_t* pe, const float* rope_row,
+                      bool fp8, float scale, uint8_t* dst) {
+  float x[kNope];
+  for (int i = 0; i < kNope; ++i) x[i] = bf16_to_f32(nope[i]);
+  encode_latent_row(x, pe, rope_row, fp8, scale, dst);
 }
 
 }  // namespace
@@ -231,6 +239,61 @@ int mla_oracle_run(const uint16_t* q_nope, int64_t qn_st, int64_t qn_sh,
     }
     build_latent_row(kv_c + t * kv_st, k_pe + t * kp_st, rope_row, kv_fp8,
                      kv_fp8 ? *kv_scale : 1.0f, kc + slot * kv_row_bytes);
+  }
+  if (status != nullptr) *status |= st;
+  return 0;
+}
+
+// Latent query rows from the absorption product (the query side of the
+// epilogue with its producer folded in).  For every token t and head h:
+//   ql[j] = sum_k q_nope_c[t, h, k] * w_uk[h, j, k],  j < 512, k < 128
+// accumulated in double precision in k order (every bf16 x bf16 product is
+// exact in double; the running sum carries 53 bits) and rounded once to
+// fp32; then the row [ql | rope(q_pe[t, h])] is encoded like every other
+// query row.
+//   q_nope_c [T,H,128] bf16 at (qc_st, qc_sh); w_uk [H,512,128] bf16 contiguous
+//   q_pe [T,H,64] at (qp_st, qp_sh); positions / cos_sin / q_scale as in mla_oracle_run
+//   q_out [T,H,576] contiguous, bf16 or e4m3 (flag Q_FP8).
+// flags: ROPE, Q_FP8 only.  Returns 0, or 1 for an unusable argument.
+int mla_oracle_absorb_run(const uint16_t* q_nope_c, int64_t qc_st, int64_t qc_sh, const uint16_t* w_uk,
+                          const uint16_t* q_pe, int64_t qp_st, int64_t qp_sh, const int32_t* positions,
+                          const float* cos_sin, int64_t rope_rows, const float* q_scale, int64_t T, int64_t H,
+                          uint32_t flags, void* q_out, int32_t* status) {
+  if (T < 0 || H < 1) return 1;
+  if ((flags & ~(kFlagRope | kFlagQFp8)) != 0) return 1;
+  if (T == 0) return 0;
+  const bool rope = (flags & kFlagRope) != 0;
+  const bool q_fp8 = (flags & kFlagQFp8) != 0;
+  if (rope && (positions == nullptr || cos_sin == nullptr || rope_rows < 1)) return 1;
+  if (q_fp8 && q_scale == nullptr) return 1;
+  constexpr int kIn = 128;
+  int32_t st = 0;
+  uint8_t* qo = static_cast<uint8_t*>(q_out);
+  const int64_t row_bytes = q_fp8 ? kRow : 2 * kRow;
+  float ql[kNope];
+  for (int64_t t = 0; t < T; ++t) {
+    const float* rope_row = nullptr;
+    if (rope) {
+      const int64_t pos = positions[t];
+      if (pos >= 0 && pos < rope_rows) {
+        rope_row = cos_sin + pos * kPe;
+      } else {
+        st |= kStatusPosRange;
+      }
+    }
+    for (int64_t h = 0; h < H; ++h) {
+      const uint16_t* a = q_nope_c + t * qc_st + h * qc_sh;
+      for (int j = 0; j < kNope; ++j) {
+        const uint16_t* b = w_uk + (h * kNope + j) * kIn;
+        double acc = 0.0;
+        for (int k = 0; k < kIn; ++k) {
+          acc += static_cast<double>(bf16_to_f32(a[k])) * static_cast<double>(bf16_to_f32(b[k]));
+        }
+        ql[j] = static_cast<float>(acc);
+      }
+      encode_latent_row(ql, q_pe + t * qp_st + h * qp_sh, rope_row, q_fp8, q_fp8 ? *q_scale : 1.0f,
+                        qo + (t * H + h) * row_bytes);
+    }
   }
   if (status != nullptr) *status |= st;
   return 0;

@@ -1,0 +1,86 @@
+"""Pins for the oracle of the absorbed query rows (the query side of the
+epilogue with the absorption product folded in)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_decode_attention_10_b200 import workloads as W
+
+
+def _bits(t):
+    t = t.contiguous()
+    return t.view(torch.int16) if t.element_size() == 2 else t
+
+
+def _run(w):
+    return oracle.absorb_run(w.q_nope_c, w.w_uk, w.q_pe, w.flags, positions=w.positions, cos_sin=w.cos_sin,
+                             q_scale=w.q_scale)
+
+
+def test_identity_weights_copy_the_input():
+    """W_UK[h] = [I_128; 0]: the first 128 latent values are the input, bit
+    for bit, the other 384 are zero."""
+    w = W.make_absorb("id", 5, 3, 0, seed=1, q_nope_row=136)
+    w.w_uk.zero_()
+    for h in range(3):
+        w.w_uk[h, :128, :] = torch.eye(128, dtype=torch.bfloat16)
+    q, st = _run(w)
+    assert st == 0
+    assert torch.equal(_bits(q[..., :128]), _bits(w.q_nope_c))
+    assert torch.all(q[..., 128:512].float() == 0)
+    assert torch.equal(_bits(q[..., 512:]), _bits(w.q_pe))
+
+
+@pytest.mark.parametrize("flags", [0, W.FLAG_Q_FP8])
+def test_small_integer_products_match_numpy(flags):
+    """Inputs that are small integers times 2^-3 make every sum exact in
+    double, so the oracle must equal numpy's float64 matmul rounded to fp32,
+    then cast by torch to bf16 (or divided by the scale and cast to e4m3)."""
+    g = torch.Generator().manual_seed(4)
+    w = W.make_absorb("ints", 6, 4, flags, seed=2, scale=0.37)
+    w.q_nope_c.copy_((torch.randint(-8, 9, w.q_nope_c.shape, generator=g).float() / 8).to(torch.bfloat16))
+    w.w_uk.copy_((torch.randint(-8, 9, w.w_uk.shape, generator=g).float() / 8).to(torch.bfloat16))
+    q, _ = _run(w)
+    a = w.q_nope_c.double().numpy()
+    b = w.w_uk.double().numpy()
+    ql = np.einsum("thk,hjk->thj", a, b)
+    ql32 = torch.from_numpy(ql.astype(np.float32))
+    if flags & W.FLAG_Q_FP8:
+        exp = (ql32 / torch.full_like(ql32, 0.37)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        assert torch.equal(q[..., :512], exp)
+    else:
+        assert torch.equal(_bits(q[..., :512]), _bits(ql32.to(torch.bfloat16)))
+
+
+@pytest.mark.parametrize("flags", [W.FLAG_ROPE, W.FLAG_ROPE | W.FLAG_Q_FP8])
+def test_pe_half_equals_the_epilogue_oracle(flags):
+    """The rotated pe half of an absorbed row is the epilogue's pe half for
+    the same q_pe, position and scale."""
+    w = W.make_absorb("pe", 7, 5, flags, seed=6, rope_rows=512, scale=0.05)
+    q, _ = _run(w)
+    e = W.make("pe_e", 7, 5, flags, seed=6, num_blocks=1, rope_rows=512, scale=0.05)
+    e.q_pe.copy_(w.q_pe)
+    e.positions.copy_(w.positions)
+    qe, _ = oracle.run(e.q_nope, e.q_pe, e.kv_c, e.k_pe, e.slot_mapping, e.cache, e.flags,
+                       positions=e.positions, cos_sin=e.cos_sin, q_scale=e.q_scale, kv_scale=e.kv_scale)
+    assert torch.equal(_bits(q[..., 512:]), _bits(qe[..., 512:]))
+
+
+def test_general_inputs_within_fp32_rounding_of_numpy():
+    w = W.make_absorb("gen", 9, 3, 0, seed=8)
+    q, _ = _run(w)
+    ql = np.einsum("thk,hjk->thj", w.q_nope_c.double().numpy(), w.w_uk.double().numpy())
+    got = q[..., :512].double().numpy()
+    ulp = np.abs(ql) * 2.0 ** -8 + 1e-30
+    assert np.all(np.abs(got - ql) <= ulp)
+
+
+def test_zero_tokens_and_bad_flags():
+    w = W.make_absorb("z", 0, 2, 0, seed=1)
+    q, st = _run(w)
+    assert q.shape == (0, 2, 576) and st == 0
+    w = W.make_absorb("f", 2, 2, 0, seed=1)
+    with pytest.raises(ValueError):
+        oracle.absorb_run(w.q_nope_c, w.w_uk, w.q_pe, W.FLAG_KV_FP8)
