@@ -34,6 +34,7 @@ MLA_FLAG_FORCE_ROWS = 32
 
 MLA_STATUS_SLOT_RANGE = 1
 MLA_STATUS_POS_RANGE = 2
+MLA_STATUS_TIMEOUT = 4
 
 MLA_MODE_SPLIT = 1
 MLA_MODE_ROWS = 2
@@ -93,6 +94,9 @@ def lib() -> ctypes.CDLL:
         L.mla_harness_empty.argtypes = [i64, i32, u32, vp]
         L.mla_harness_consume.restype = ctypes.c_int
         L.mla_harness_consume.argtypes = [vp, vp, vp, i64, i64, i64, u32, vp, vp]
+        L.mla_absorb_launch.restype = ctypes.c_int
+        L.mla_absorb_launch.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, vp, i64, i64, u32,
+                                        vp, vp, vp]
         L.mla_harness_div_check.restype = ctypes.c_int
         L.mla_harness_div_check.argtypes = [ctypes.c_float, u64, u64, vp, vp]
         _lib = L
@@ -156,6 +160,14 @@ def mla_harness_consume(q_out, cache, slot_mapping, T, H, cache_rows, flags, sco
 
 def mla_harness_div_check(scale: float, first: int, count: int, result, stream) -> int:
     return lib().mla_harness_div_check(scale, first, count, result, stream)
+
+
+def mla_absorb_launch(q_nope_c, q_nope_c_stride_t, q_nope_c_stride_h, w_uk, q_pe, q_pe_stride_t, q_pe_stride_h,
+                      positions, cos_sin, rope_rows, q_scale, T, H, flags, q_out, status, stream) -> int:
+    """The query rows from the absorption product (include/mla_absorb.h); returns the mla_status code."""
+    return lib().mla_absorb_launch(q_nope_c, q_nope_c_stride_t, q_nope_c_stride_h, w_uk, q_pe, q_pe_stride_t,
+                                   q_pe_stride_h, positions, cos_sin, rope_rows, q_scale, T, H, flags, q_out,
+                                   status, stream)
 
 
 # ---- torch convenience ------------------------------------------------------------------
@@ -232,6 +244,16 @@ def fused_mla_decode_q_concat_kv_cache_insert(
     if rc != MLA_OK:
         raise MlaError(rc, "mla_epilogue_launch")
     return q_out
+
+
+def launch_absorb_workload(w, q_out: torch.Tensor, *, status: Optional[torch.Tensor] = None,
+                           extra_flags: int = 0, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Launch mla_absorb_launch on a device-resident ``workloads.AbsorbWorkload``."""
+    return mla_absorb_launch(
+        _dptr(w.q_nope_c), w.q_nope_c.stride(0), w.q_nope_c.stride(1), _dptr(w.w_uk),
+        _dptr(w.q_pe), w.q_pe.stride(0), w.q_pe.stride(1), _dptr(w.positions), _dptr(w.cos_sin),
+        w.cos_sin.shape[0] if w.cos_sin is not None else 0, _dptr(w.q_scale), w.T, w.H,
+        w.flags | extra_flags, _dptr(q_out), _dptr(status), _stream_handle(stream))
 
 
 def launch_workload(w, q_out: torch.Tensor, *, status: Optional[torch.Tensor] = None,

@@ -13,7 +13,7 @@ from mla_decode_attention_10_b200 import build as B
 from mla_decode_attention_10_b200 import epilogue as E
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADERS = [os.path.join(ROOT, "include", h) for h in ("mla_epilogue.h", "mla_harness.h")]
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("mla_epilogue.h", "mla_harness.h", "mla_absorb.h")]
 
 
 @pytest.fixture(scope="module")
@@ -201,3 +201,30 @@ def test_harness_validation(lib, kw, code):
     assert E.mla_harness_consume(None, A, A, 4, 16, 64, 0, A, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_consume(A + 8, A, A, 4, 16, 64, 0, A, None) == E.MLA_ERR_ALIGNMENT
     assert E.mla_harness_consume(A, A, A, 0, 16, 64, 0, None, None) == E.MLA_OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(flags=E.MLA_FLAG_KV_FP8), E.MLA_ERR_UNSUPPORTED),
+    (dict(T=-1), E.MLA_ERR_INVALID_ARG),
+    (dict(H=0), E.MLA_ERR_INVALID_ARG),
+    (dict(H=65536), E.MLA_ERR_INVALID_ARG),
+    (dict(q_nope_c=None), E.MLA_ERR_INVALID_ARG),
+    (dict(w_uk=None), E.MLA_ERR_INVALID_ARG),
+    (dict(q_out=None), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_ROPE, positions=None), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_Q_FP8, q_scale=None), E.MLA_ERR_INVALID_ARG),
+    (dict(q_nope_c=A + 8), E.MLA_ERR_ALIGNMENT),
+    (dict(w_uk=A + 2), E.MLA_ERR_ALIGNMENT),
+    (dict(q_out=A + 4), E.MLA_ERR_ALIGNMENT),
+    (dict(q_nope_c_stride_h=132), E.MLA_ERR_ALIGNMENT),
+    (dict(q_pe=A + 1), E.MLA_ERR_ALIGNMENT),
+])
+def test_absorb_validation(lib, kw, code):
+    args = dict(q_nope_c=A, q_nope_c_stride_t=16 * 128, q_nope_c_stride_h=128, w_uk=A, q_pe=A,
+                q_pe_stride_t=16 * 64, q_pe_stride_h=64, positions=A, cos_sin=A, rope_rows=8, q_scale=A,
+                T=4, H=16, flags=0, q_out=A, status=None, stream=None)
+    args.update(kw)
+    assert E.mla_absorb_launch(**args) == code
+    args.update(T=0, q_nope_c=None, w_uk=None, q_out=None)
+    if code != E.MLA_ERR_UNSUPPORTED and kw.get("H", 1) >= 1 and kw.get("H", 1) < 65536 and kw.get("T", 0) >= 0:
+        assert E.mla_absorb_launch(**args) == E.MLA_OK
