@@ -420,11 +420,24 @@ def run_ours(args, rank, world, local_rank):
     e2e = run_e2e(args, w0, stream, device, world)
 
     # ---- sweep of the other sizes (their own bench lines are not printed; this is context)
+    # the headline is measured; what follows is context, and an error in it is
+    # reported in the line rather than losing the line
     sweep = []
+    context_errors = []
     if not args.no_sweep:
         for name in sweep_names(args.workload):
-            sweep.append(sweep_one(name, E, stream, device, peak, epilogue_step, floor_step, measure))
+            try:
+                sweep.append(sweep_one(name, E, stream, device, peak, epilogue_step, floor_step, measure))
+            except Exception as exc:  # noqa: BLE001
+                context_errors.append(f"{name}: {type(exc).__name__}: {str(exc).splitlines()[0][:200]}")
             torch.cuda.empty_cache()
+
+    absorb = None
+    if not args.no_sweep:
+        try:
+            absorb = absorb_measure(E, stream, device, peak)
+        except Exception as exc:  # noqa: BLE001
+            context_errors.append(f"absorbed_query: {type(exc).__name__}: {str(exc).splitlines()[0][:200]}")
 
     line = {
         "metric": METRIC, "value": round(us, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -459,6 +472,10 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
         "sweep": sweep,
     }
+    if absorb is not None:
+        line["absorbed_query"] = absorb
+    if context_errors:
+        line["context_errors"] = context_errors
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args.workload)
     return line
@@ -584,28 +601,108 @@ def producer_consumer_chain(ds, E, stream, device, n, warmup):
     return out
 
 
+def absorb_measure(E, stream, device, peak_gbs):
+    """The query side with the absorption product folded in (tcgen05 kernel)
+    at T=8192, H=16, RoPE, e4m3, against the same work unfused: a cuBLAS
+    batched matmul writing the 512-wide product, then the epilogue (which
+    also writes the cache rows)."""
+    peak_tf = None
+    try:
+        peak_tf = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        peak_tf = 1590.0
+    sets = []
+    for k in range(2):
+        w = W.make_absorb("absorb_t8192_h16_rope_fp8", 8192, 16, W.FLAG_ROPE | W.FLAG_Q_FP8, seed=k,
+                          rope_rows=131072).to(device)
+        q_out = torch.empty((w.T, w.H, W.ROW), dtype=torch.uint8, device=device)
+        sets.append((w, q_out))
+    w0 = sets[0][0]
+
+    def fused(i):
+        w, q = sets[i % 2]
+        assert E.launch_absorb_workload(w, q, stream=stream) == E.MLA_OK
+
+    n = 20
+    r = GraphRunner(fused, n, stream)
+    r.replay()
+    torch.cuda.synchronize()
+    us = min(timed(r, device) for _ in range(3)) * 1e3 / n
+    del r
+    # unfused: torch.bmm (cuBLAS) for the product, then the epilogue on it
+    e_sets = []
+    for k, (w, q) in enumerate(sets):
+        ew = W.make("absorb_unfused", w.T, w.H, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8, seed=k,
+                    num_blocks=16384, rope_rows=131072).to(device)
+        ql = torch.empty((w.H, w.T, W.NOPE), dtype=torch.bfloat16, device=device)
+        ew.q_nope = ql.transpose(0, 1)
+        ew.q_pe = w.q_pe
+        e_sets.append((w, ew, ql, torch.empty((w.T, w.H, W.ROW), dtype=torch.uint8, device=device)))
+
+    def bmm_only(i):
+        w, _, ql, _ = e_sets[i % 2]
+        with torch.cuda.stream(stream):
+            torch.bmm(w.q_nope_c.transpose(0, 1), w.w_uk.transpose(1, 2), out=ql)
+
+    def unfused(i):
+        bmm_only(i)
+        _, ew, _, q = e_sets[i % 2]
+        assert E.launch_workload(ew, q, stream=stream) == E.MLA_OK
+
+    # cuBLAS creates its handle and workspace on first use, which cannot happen inside a graph capture
+    bmm_only(0)
+    torch.cuda.synchronize()
+    out = {}
+    for key, fn in (("bmm_us", bmm_only), ("bmm_plus_epilogue_us", unfused)):
+        g = GraphRunner(fn, n, stream)
+        g.replay()
+        torch.cuda.synchronize()
+        out[key] = round(min(timed(g, device) for _ in range(3)) * 1e3 / n, 3)
+        del g
+    gbs = w0.algorithmic_bytes() / (us * 1e-6) / 1e9
+    tfs = w0.flops() / (us * 1e-6) / 1e12
+    return {"workload": "absorb_t8192_h16_rope_fp8",
+            "recipe": "T=8192 H=16: q_nope_c [8192,16,128] and q_pe bf16 N(0,1), W_UK [16,512,128] N(0,1/128), "
+                      "RoPE (131072-row table), e4m3 scale 0.05; two input sets, seeds 0 and 1",
+            "us_per_call": round(us, 3), "bytes_per_call": w0.algorithmic_bytes(), "flops_per_call": w0.flops(),
+            "gbs": round(gbs, 1), "frac_hbm": round(gbs / peak_gbs, 4), "tflops": round(tfs, 1),
+            "frac_tensor": round(tfs / peak_tf, 4), "bound": "hbm" if gbs / peak_gbs > tfs / peak_tf else "tensor",
+            **out}
+
+
 def run_e2e(args, w0, stream, device, world):
     """Same metric through the user-facing call, with host buffers: every step
     copies its inputs from pinned host memory, runs the epilogue and copies
-    q_out back, all on one stream, timed with CUDA events."""
+    q_out back, all on one stream, timed with CUDA events.  The per-step
+    inputs (q_nope, q_pe, kv_c, k_pe, slot_mapping, positions) sit in one
+    pinned staging buffer at 16-byte aligned offsets, so each step is one
+    host-to-device copy, the call, and one device-to-host copy."""
     from mla_decode_attention_10_b200 import epilogue as E
-    host = {k: getattr(w0, k).contiguous().pin_memory()
-            for k in ("q_nope", "q_pe", "kv_c", "k_pe", "slot_mapping", "positions")
-            if getattr(w0, k) is not None}
-    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    parts = [(k, getattr(w0, k).contiguous()) for k in ("q_nope", "q_pe", "kv_c", "k_pe", "slot_mapping", "positions")
+             if getattr(w0, k) is not None]
+    offsets, total = {}, 0
+    for k, v in parts:
+        offsets[k] = total
+        total += -(-v.numel() * v.element_size() // 16) * 16
+    host = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for k, v in parts:
+        n = v.numel() * v.element_size()
+        host[offsets[k]:offsets[k] + n].copy_(v.view(-1).view(torch.uint8))
+    dbuf = torch.empty(total, dtype=torch.uint8, device=device)
+    dev = {k: dbuf[offsets[k]:offsets[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+           for k, v in parts}
     cache = w0.cache.to(device)
     cos_sin = w0.cos_sin.to(device) if w0.cos_sin is not None else None
     qs = w0.q_scale.to(device) if w0.q_scale is not None else None
     ks = w0.kv_scale.to(device) if w0.kv_scale is not None else None
     q_out = torch.empty((w0.T, w0.H, W.ROW), dtype=w0.q_out_dtype(), device=device)
     q_host = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    h2d = sum(v.numel() * v.element_size() for _, v in parts)
     d2h = q_host.numel() * q_host.element_size()
 
     def step():
         with torch.cuda.stream(stream):
-            for k, v in host.items():
-                dev[k].copy_(v, non_blocking=True)
+            dbuf.copy_(host, non_blocking=True)
             E.fused_mla_decode_q_concat_kv_cache_insert(
                 dev["q_nope"], dev["q_pe"], dev["kv_c"], dev["k_pe"], cache, dev["slot_mapping"],
                 positions=dev.get("positions"), cos_sin=cos_sin, q_scale=qs, kv_scale=ks,
@@ -627,8 +724,8 @@ def run_e2e(args, w0, stream, device, world):
     ms = max_over_ranks(e0.elapsed_time(e1), device)
     return {"value": round(job_us_per_call(ms, k, world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": k,
-            "path": "epilogue.fused_mla_decode_q_concat_kv_cache_insert, pinned host <-> device copies on the "
-                    "launch stream"}
+            "path": "epilogue.fused_mla_decode_q_concat_kv_cache_insert; inputs from one pinned staging buffer "
+                    "(one host-to-device copy), q_out back to pinned host memory, all on the launch stream"}
 
 
 # ---------------------------------------------------------------------------------------
