@@ -1,23 +1,29 @@
 // mla_absorb.cu -- latent query rows straight from the absorption product, on
 // the tcgen05 tensor cores (contract in mla_absorb.h).
 //
-// One CTA of four warps computes a 128-token x 256-column tile of one head:
-//   * the A tile (q_nope_c: 128 tokens x 128) and the B tile (w_uk: 256 latent
-//     rows x 128) arrive by TMA with the 128-byte swizzle, as two 64-wide
-//     column slabs each, on one mbarrier; the weights are requested before
-//     the kernel waits for the upstream grid, the query after;
-//   * one thread issues eight M=128, N=256, K=16 tcgen05.mma (bf16 in, fp32
-//     accumulate) into 256 TMEM columns and commits them to a second mbarrier;
-//   * each warp reads its 32 TMEM lanes (tokens) back with tcgen05.ld, 32
-//     columns at a time, and writes them encoded (bf16, or e4m3 of x / scale)
-//     straight into q_out's row layout;
-//   * the CTAs of the second column tile also rotate and write the 64 pe
-//     values of their 128 tokens, one RoPE pair per lane, while the tensor
-//     cores run.
-// The weights of a head are 128 KB and stay in L2 across tiles; the two column
-// tiles of one token tile are adjacent in the grid so the A tile is read from
-// HBM once.  Every wait is bounded: on timeout the kernel sets a status bit,
-// waits (bounded) for what it issued, frees its TMEM and returns.
+// A persistent kernel, one CTA per SM, that takes a contiguous run of
+// 128-token x 256-column tiles in (head, column half, token tile) order, so a
+// head's weights are loaded once for many token tiles.  Its warps have roles:
+//   * warp 0 (TMA): per tile, the A tile (q_nope_c: 128 tokens x 128) into a
+//     two-stage ring and, when the (head, column half) changes, the B tile
+//     (w_uk: 256 latent rows x 128), both with the 128-byte swizzle; the
+//     weights before waiting for the upstream grid, the queries after;
+//   * warp 1 (MMA): allocates 512 TMEM columns and per tile issues eight
+//     M=128, N=256, K=16 tcgen05.mma (bf16 in, fp32 accumulate) into one of
+//     two 256-column accumulators, committing to the A stage's "empty" and
+//     the accumulator's "full" barrier;
+//   * warps 2..9 (epilogue): the warp of TMEM lane quarter w mod 4 and column
+//     half (w - 2) / 4 reads its 32 tokens x 128 columns with tcgen05.ld,
+//     encodes them (bf16, or e4m3 of x / scale) into a staging tile with the
+//     128-byte swizzle, frees the accumulator, and one thread per half sends
+//     each 128-byte column slab out with one bulk tensor store, so HBM sees
+//     whole-line writes;
+//   * warps 10..13 (rotary): per tile, the 64 pe values of 64 of its tokens,
+//     two threads per token, every load issued before any is used.
+// The loads of tile i+1, its MMAs and the epilogue of tile i overlap.  Every
+// wait is bounded: on timeout the kernel sets a status bit, every role stops,
+// the copies in flight are waited for (bounded), TMEM is freed and the kernel
+// returns.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -39,12 +45,17 @@ constexpr int kNope = 512;
 constexpr int kPe = 64;
 constexpr int kHalfPe = 32;
 constexpr int kRow = 576;
-constexpr int kThreads = 128;
+constexpr int kTmaWarp = 0, kMmaWarp = 1, kEpiWarp0 = 2, kEpiWarps = 8, kPeWarp0 = 10, kPeWarps = 4;
+constexpr int kThreads = 32 * (kPeWarp0 + kPeWarps);  // 448
+constexpr int kStages = 2;                            // A ring
 constexpr uint32_t kSlabA = kM * 64 * 2;     // one 64-wide column slab of A: 16 KB
 constexpr uint32_t kSlabB = kN * 64 * 2;     // one 64-wide column slab of B: 32 KB
-constexpr uint32_t kTileBytes = 2 * kSlabA + 2 * kSlabB;  // 96 KB
-constexpr uint32_t kSmemBytes = kTileBytes + 1024;        // + room to align to 1024
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kSlabC = kM * 128;        // one 128-byte column slab of the output tile: 16 KB
+constexpr uint32_t kABytes = 2 * kSlabA;                 // 32 KB
+constexpr uint32_t kBBytes = 2 * kSlabB;                 // 64 KB
+constexpr uint32_t kCBytes = 4 * kSlabC;                 // output staging, 64 KB
+constexpr uint32_t kSmemBytes = kBBytes + kStages * kABytes + kCBytes + 1024;
+constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 constexpr uint32_t kWaitSpins = 1u << 24;
 
 struct Params {
@@ -57,6 +68,8 @@ struct Params {
   int32_t T, H;
   uint8_t* q_out;
   int32_t* status;
+  int32_t pe_vec;   // q_pe rows may be read as 16-byte vectors
+  int32_t tab_vec;  // cos_sin rows may be read as 16-byte vectors
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -112,6 +125,9 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b
       : "memory");
 }
 
+// tcgen05.ld of 32 columns of this warp's 32 TMEM lanes, then its wait; the
+// wait names the loaded registers, so no use of them can be scheduled
+// before it
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
@@ -122,15 +138,41 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr)
       : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                 "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
+                 "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
 }
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// 32 accumulator values (columns c..c+31 of one token row) -> q_out.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// 32 accumulator values (columns col..col+31 of tile row r), encoded, into
+// the output staging tile: 128-byte column slabs of 128 rows each
+// (kSlabCols columns), with the 128-byte swizzle the bulk tensor store
+// expects (16-byte piece j of row r at position j ^ (r mod 8)).  Eight
+// consecutive rows thus cover all 32 banks for one piece index.
 template <bool QF8, bool FAST>
-__device__ __forceinline__ void store_chunk(uint8_t* row, int col, const uint32_t (&v)[32], const Divisor& d) {
+__device__ __forceinline__ void stage_chunk(uint32_t sC, int r, int col, const uint32_t (&v)[32], const Divisor& d) {
+  constexpr int kSlabCols = QF8 ? 128 : 64;
+  const uint32_t rowbase = sC + static_cast<uint32_t>(col / kSlabCols) * kSlabC + static_cast<uint32_t>(r) * 128u;
+  const uint32_t j0 = static_cast<uint32_t>((col % kSlabCols) * (QF8 ? 1 : 2) / 16);
+  const uint32_t sw = static_cast<uint32_t>(r & 7);
   if constexpr (QF8) {
     uint32_t w[8];
 #pragma unroll
@@ -139,158 +181,359 @@ __device__ __forceinline__ void store_chunk(uint8_t* row, int col, const uint32_
       const uint32_t hi = e4m3x2_of_f32<FAST>(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]), d);
       w[i] = lo | (hi << 16);
     }
-    uint4* dst = reinterpret_cast<uint4*>(row + col);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      st_shared_v4(rowbase + (((j0 + q) ^ sw) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   } else {
     uint32_t w[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    uint4* dst = reinterpret_cast<uint4*>(row + 2 * col);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    for (int q = 0; q < 4; ++q)
+      st_shared_v4(rowbase + (((j0 + q) ^ sw) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   }
 }
 
-// The 64 rotary values of tokens m0..m0+127 of head h: warp w takes rows
-// w, w+4, ...; lane i the pair (i, i+32).
+// The 64 rotary values of 64 of a tile's tokens: the tile of column half nt
+// covers tokens m0 + 64 nt .. m0 + 64 nt + 63, two threads (tid 2j, 2j+1)
+// per token, each 16 of the 32 rotation pairs (i, i+32).  Every thread
+// issues all of its loads (its q_pe values and its cos and sin entries, as
+// 16-byte vectors when the host found them aligned) before it uses any, so
+// a tile costs about two memory round trips (position, then table).
 template <bool QF8, bool ROPE, bool FAST>
-__device__ __forceinline__ void pe_rows(const Params& p, int m0, int h, const Divisor& d) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  for (int r = warp; r < kM; r += kThreads / 32) {
-    const int t = m0 + r;
-    if (t >= p.T) break;
-    float c = 1.0f, s = 0.0f;
-    bool on = false;
-    if constexpr (ROPE) {
-      const int64_t pos = __ldg(p.positions + t);
-      if (pos >= 0 && pos < p.rope_rows) {
-        const float* tab = p.cos_sin + pos * kPe;
-        c = __ldg(tab + lane);
-        s = __ldg(tab + kHalfPe + lane);
-        on = true;
-      } else if (lane == 0 && h == 0) {
-        report(p.status, MLA_STATUS_POS_RANGE);
-      }
-    }
-    const uint16_t* pe = p.q_pe + static_cast<int64_t>(t) * p.qp_st + static_cast<int64_t>(h) * p.qp_sh;
-    const uint32_t raw = static_cast<uint32_t>(__ldcg(pe + lane)) | (static_cast<uint32_t>(__ldcg(pe + kHalfPe + lane)) << 16);
-    float a = bf16_lo(raw), b = bf16_hi(raw);
-    bool rotated = false;
-    if (ROPE && on) {
-      float ya, yb;
-      rope_pair(a, b, c, s, ya, yb);
-      a = ya;
-      b = yb;
-      rotated = true;
-    }
-    uint8_t* row = p.q_out + (static_cast<int64_t>(t) * p.H + h) * (QF8 ? kRow : 2 * kRow);
-    if constexpr (QF8) {
-      const uint32_t e = e4m3x2_of_f32<FAST>(a, b, d);
-      row[kNope + lane] = static_cast<uint8_t>(e & 0xffu);
-      row[kNope + kHalfPe + lane] = static_cast<uint8_t>((e >> 8) & 0xffu);
-    } else {
-      const uint32_t o = rotated ? pack_bf16x2(a, b) : raw;
-      uint16_t* r16 = reinterpret_cast<uint16_t*>(row);
-      r16[kNope + lane] = static_cast<uint16_t>(o & 0xffffu);
-      r16[kNope + kHalfPe + lane] = static_cast<uint16_t>(o >> 16);
-    }
-  }
-}
-
-template <bool QF8, bool ROPE, bool FAST>
-__device__ __forceinline__ void tile(const CUtensorMap* tmA, const CUtensorMap* tmB, const Params& p,
-                                     uint32_t sbase, uint32_t bar_tma, uint32_t bar_mma, uint32_t tmem,
-                                     volatile uint32_t* fail, const Divisor& d) {
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int m0 = static_cast<int>(blockIdx.x >> 1) * kM;
-  const int nt = static_cast<int>(blockIdx.x & 1u);
-  const int n0 = nt * kN;
-  const int h = static_cast<int>(blockIdx.y);
-  const uint32_t sA = sbase;                  // two 16 KB slabs: k 0..63, 64..127
-  const uint32_t sB = sbase + 2 * kSlabA;     // two 32 KB slabs
-
-  if (threadIdx.x == 0) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_tma), "r"(kTileBytes)
-                 : "memory");
-    // weights do not depend on the upstream kernel
-    tma_load_3d(sB, tmB, 0, n0, h, bar_tma);
-    tma_load_3d(sB + kSlabB, tmB, 64, n0, h, bar_tma);
-    pdl_wait();
-    tma_load_3d(sA, tmA, 0, h, m0, bar_tma);
-    tma_load_3d(sA + kSlabA, tmA, 64, h, m0, bar_tma);
-    if (wait_phase(bar_tma, 0)) {
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+__device__ __forceinline__ void pe_part(const Params& p, int m0, int nt, int h, int tid, const Divisor& d) {
+  const int t = m0 + 64 * nt + (tid >> 1);
+  if (t >= p.T) return;
+  const int i0 = (tid & 1) * 16;  // first rotation pair of this thread
+  const uint16_t* pe = p.q_pe + static_cast<int64_t>(t) * p.qp_st + static_cast<int64_t>(h) * p.qp_sh;
+  int32_t pos = 0;
+  if constexpr (ROPE) pos = __ldg(p.positions + t);
+  uint32_t ra[8], rb[8];  // bf16 pairs: first-half values a_i and second-half values b_i = pe[i + 32]
+  if (p.pe_vec) {
+    const uint4* va = reinterpret_cast<const uint4*>(pe + i0);
+    const uint4* vb = reinterpret_cast<const uint4*>(pe + kHalfPe + i0);
+    const uint4 a0 = __ldcg(va), a1 = __ldcg(va + 1), b0 = __ldcg(vb), b1 = __ldcg(vb + 1);
+    ra[0] = a0.x; ra[1] = a0.y; ra[2] = a0.z; ra[3] = a0.w; ra[4] = a1.x; ra[5] = a1.y; ra[6] = a1.z; ra[7] = a1.w;
+    rb[0] = b0.x; rb[1] = b0.y; rb[2] = b0.z; rb[3] = b0.w; rb[4] = b1.x; rb[5] = b1.y; rb[6] = b1.z; rb[7] = b1.w;
+  } else {
 #pragma unroll
-      for (int j = 0; j < kK / 16; ++j) {
-        // K step j: slab j/4, 32 bytes (16 bf16) further per step inside the 128-byte row
-        const uint32_t off = static_cast<uint32_t>(j & 3) * 32u;
-        const uint64_t a = smem_desc_sw128(sA + static_cast<uint32_t>(j >> 2) * kSlabA + off);
-        const uint64_t b = smem_desc_sw128(sB + static_cast<uint32_t>(j >> 2) * kSlabB + off);
-        mma_bf16(tmem, a, b, j > 0 ? 1u : 0u);
-      }
-    } else {
-      *fail = 1u;
-      report(p.status, MLA_STATUS_TIMEOUT);
-      (void)wait_phase(bar_tma, 0);  // the copies may still land: give them one more bounded wait
+    for (int k = 0; k < 8; ++k) {
+      ra[k] = static_cast<uint32_t>(__ldcg(pe + i0 + 2 * k)) | (static_cast<uint32_t>(__ldcg(pe + i0 + 2 * k + 1)) << 16);
+      rb[k] = static_cast<uint32_t>(__ldcg(pe + kHalfPe + i0 + 2 * k)) |
+              (static_cast<uint32_t>(__ldcg(pe + kHalfPe + i0 + 2 * k + 1)) << 16);
     }
-    // arrives once every MMA issued above has completed (at once if none was)
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_mma)
-                 : "memory");
   }
-
-  if (nt == 1) {
-    pdl_wait();  // q_pe comes from the upstream kernel
-    pe_rows<QF8, ROPE, FAST>(p, m0, h, d);
+  float c[16], s[16];
+  bool on = false;
+  if constexpr (ROPE) {
+    on = pos >= 0 && pos < p.rope_rows;
+    if (!on && h == 0 && (tid & 1) == 0) report(p.status, MLA_STATUS_POS_RANGE);
+    if (on) {
+      const float* tab = p.cos_sin + static_cast<int64_t>(pos) * kPe;
+      if (p.tab_vec) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 cv = __ldg(reinterpret_cast<const float4*>(tab + i0) + k);
+          const float4 sv = __ldg(reinterpret_cast<const float4*>(tab + kHalfPe + i0) + k);
+          c[4 * k] = cv.x; c[4 * k + 1] = cv.y; c[4 * k + 2] = cv.z; c[4 * k + 3] = cv.w;
+          s[4 * k] = sv.x; s[4 * k + 1] = sv.y; s[4 * k + 2] = sv.z; s[4 * k + 3] = sv.w;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          c[k] = __ldg(tab + i0 + k);
+          s[k] = __ldg(tab + kHalfPe + i0 + k);
+        }
+      }
+    }
   }
-
-  // warp-uniform: tcgen05.ld below is a whole-warp instruction
-  const bool ok = __all_sync(0xffffffffu, wait_phase(bar_mma, 0));
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (!ok) {
-    if (lane == 0) report(p.status, MLA_STATUS_TIMEOUT);
-    return;
+  float ya[16], yb[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float a = (k & 1) ? bf16_hi(ra[k >> 1]) : bf16_lo(ra[k >> 1]);
+    const float b = (k & 1) ? bf16_hi(rb[k >> 1]) : bf16_lo(rb[k >> 1]);
+    ya[k] = a;
+    yb[k] = b;
+    if (ROPE && on) rope_pair(a, b, c[k], s[k], ya[k], yb[k]);
   }
-  if (__any_sync(0xffffffffu, *fail != 0u)) return;
-  const int r = warp * 32 + lane;  // TMEM lane = accumulator row = token m0 + r
-  const int t = m0 + r;
   uint8_t* row = p.q_out + (static_cast<int64_t>(t) * p.H + h) * (QF8 ? kRow : 2 * kRow);
+  if constexpr (QF8) {
+    uint32_t wa[4], wb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      wa[j] = e4m3x2_of_f32<FAST>(ya[4 * j], ya[4 * j + 1], d) | (e4m3x2_of_f32<FAST>(ya[4 * j + 2], ya[4 * j + 3], d) << 16);
+      wb[j] = e4m3x2_of_f32<FAST>(yb[4 * j], yb[4 * j + 1], d) | (e4m3x2_of_f32<FAST>(yb[4 * j + 2], yb[4 * j + 3], d) << 16);
+    }
+    *reinterpret_cast<uint4*>(row + kNope + i0) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    *reinterpret_cast<uint4*>(row + kNope + kHalfPe + i0) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+  } else {
+    uint32_t wa[8], wb[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      // an unrotated value keeps its bits (NaN payloads included)
+      wa[j] = (ROPE && on) ? pack_bf16x2(ya[2 * j], ya[2 * j + 1]) : ra[j];
+      wb[j] = (ROPE && on) ? pack_bf16x2(yb[2 * j], yb[2 * j + 1]) : rb[j];
+    }
+    uint4* da = reinterpret_cast<uint4*>(row + 2 * (kNope + i0));
+    uint4* db = reinterpret_cast<uint4*>(row + 2 * (kNope + kHalfPe + i0));
+    da[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    da[1] = make_uint4(wa[4], wa[5], wa[6], wa[7]);
+    db[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    db[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
+  }
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag) {
+  for (uint32_t i = 0; i < kWaitSpins; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (*abort_flag != 0u) return false;
+  }
+  return false;
+}
+
+// barrier `id` over `n` threads, returning the AND of `pred` over them
+__device__ __forceinline__ bool bar_and(int id, int n, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
+      : "memory");
+  return out != 0u;
+}
+
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// Tile order: (head, column half, token tile), token tile fastest.
+struct TileCoord {
+  int h, nt, m0;
+};
+
+__device__ __forceinline__ TileCoord tile_at(int idx, int mt) {
+  TileCoord c;
+  const int g = idx / mt;
+  c.m0 = (idx - g * mt) * kM;
+  c.h = g >> 1;
+  c.nt = g & 1;
+  return c;
+}
+
+struct Bars {
+  uint64_t a_full[kStages], a_empty[kStages];
+  uint64_t b_full, b_empty;
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_done;
+};
+
+template <bool QF8, bool ROPE, bool FAST>
+__device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmC,
+                                    const Params& p, uint32_t sbase, const Bars& bars, uint32_t tmem,
+                                    volatile uint32_t* abort_flag, const Divisor& d) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int mt = (p.T + kM - 1) / kM;
+  const int tiles = 2 * p.H * mt;
+  const int per = tiles / static_cast<int>(gridDim.x);
+  const int rem = tiles - per * static_cast<int>(gridDim.x);
+  const int bx = static_cast<int>(blockIdx.x);
+  const int first = bx * per + (bx < rem ? bx : rem);
+  const int count = per + (bx < rem ? 1 : 0);
+  const uint32_t sB = sbase;
+  const uint32_t sA = sbase + kBBytes;
+  const uint32_t sC = sA + kStages * kABytes;
+
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      bool waited = false;
+      int group = -1, groups = 0, issued = 0;
+      for (int i = 0; i < count && *abort_flag == 0u; ++i) {
+        const TileCoord c = tile_at(first + i, mt);
+        const int g = c.h * 2 + c.nt;
+        if (g != group) {
+          if (groups > 0 && !wait_or_abort(smem_u32(&bars.b_empty), static_cast<uint32_t>(groups - 1) & 1u, abort_flag)) {
+            *abort_flag = 1u;
+            report(p.status, MLA_STATUS_TIMEOUT);
+            break;
+          }
+          const uint32_t bf = smem_u32(&bars.b_full);
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bf), "r"(kBBytes) : "memory");
+          tma_load_3d(sB, tmB, 0, c.nt * kN, c.h, bf);
+          tma_load_3d(sB + kSlabB, tmB, 64, c.nt * kN, c.h, bf);
+          group = g;
+          ++groups;
+        }
+        const int st = i % kStages;
+        const int use = i / kStages;
+        if (use > 0 && !wait_or_abort(smem_u32(&bars.a_empty[st]), static_cast<uint32_t>(use - 1) & 1u, abort_flag)) {
+          *abort_flag = 1u;
+          report(p.status, MLA_STATUS_TIMEOUT);
+          break;
+        }
+        if (!waited) {
+          pdl_wait();  // the queries come from the upstream kernel
+          waited = true;
+        }
+        const uint32_t af = smem_u32(&bars.a_full[st]);
+        const uint32_t dst = sA + static_cast<uint32_t>(st) * kABytes;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(af), "r"(kABytes) : "memory");
+        tma_load_3d(dst, tmA, 0, c.h, c.m0, af);
+        tma_load_3d(dst + kSlabA, tmA, 64, c.h, c.m0, af);
+        issued = i + 1;
+      }
+      // every copy issued has landed before the CTA may end
+      for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
+        (void)wait_phase(smem_u32(&bars.a_full[i % kStages]), static_cast<uint32_t>(i / kStages) & 1u);
+      if (groups > 0) (void)wait_phase(smem_u32(&bars.b_full), static_cast<uint32_t>(groups - 1) & 1u);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      int group = -1, groups = 0;
+      for (int i = 0; i < count && *abort_flag == 0u; ++i) {
+        const TileCoord c = tile_at(first + i, mt);
+        const int g = c.h * 2 + c.nt;
+        if (g != group) {
+          if (!wait_or_abort(smem_u32(&bars.b_full), static_cast<uint32_t>(groups) & 1u, abort_flag)) {
+            *abort_flag = 1u;
+            report(p.status, MLA_STATUS_TIMEOUT);
+            break;
+          }
+          group = g;
+          ++groups;
+        }
+        const int st = i % kStages;
+        const int b = i & 1;
+        if (!wait_or_abort(smem_u32(&bars.a_full[st]), static_cast<uint32_t>(i / kStages) & 1u, abort_flag) ||
+            (i >= 2 && !wait_or_abort(smem_u32(&bars.acc_empty[b]), static_cast<uint32_t>(i / 2 - 1) & 1u, abort_flag))) {
+          *abort_flag = 1u;
+          report(p.status, MLA_STATUS_TIMEOUT);
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a0 = sA + static_cast<uint32_t>(st) * kABytes;
+        const uint32_t acc = tmem + static_cast<uint32_t>(b) * kN;
+#pragma unroll
+        for (int j = 0; j < kK / 16; ++j) {
+          const uint32_t off = static_cast<uint32_t>(j & 3) * 32u;
+          mma_bf16(acc, smem_desc_sw128(a0 + static_cast<uint32_t>(j >> 2) * kSlabA + off),
+                   smem_desc_sw128(sB + static_cast<uint32_t>(j >> 2) * kSlabB + off), j > 0 ? 1u : 0u);
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&bars.a_empty[st]))
+                     : "memory");
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&bars.acc_full[b]))
+                     : "memory");
+        bool last_of_group = (i + 1 == count);
+        if (!last_of_group) {
+          const TileCoord n = tile_at(first + i + 1, mt);
+          last_of_group = (n.h * 2 + n.nt) != g;
+        }
+        if (last_of_group)
+          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           smem_u32(&bars.b_empty))
+                       : "memory");
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32(&bars.mma_done))
+                   : "memory");
+      (void)wait_phase(smem_u32(&bars.mma_done), 0u);
+    }
+  } else if (warp < kPeWarp0) {
+    // epilogue: warp w reads TMEM lane quarter w mod 4, columns 128 hf .. 128 hf + 127
+    const int ew = warp - kEpiWarp0;
+    const int hf = ew >> 2;
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const bool issuer = (ew & 3) == 0 && lane == 0;  // issues the bulk stores of its half
+    constexpr int kSlabCols = QF8 ? 128 : 64;
+    for (int i = 0; i < count; ++i) {
+      const TileCoord c = tile_at(first + i, mt);
+      const int b = i & 1;
+      const bool ready = wait_or_abort(smem_u32(&bars.acc_full[b]), static_cast<uint32_t>(i / 2) & 1u, abort_flag);
+      // this half's previous stores have finished reading the staging tile
+      if (issuer) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      if (!bar_and(1, 32 * kEpiWarps, ready && *abort_flag == 0u)) {
+        if (lane == 0 && ew == 0) {
+          *abort_flag = 1u;
+          report(p.status, MLA_STATUS_TIMEOUT);
+        }
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t acc = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b) * kN;
 #pragma unroll 1
-  for (int c = 0; c < kN; c += 32) {
-    uint32_t v[32];
-    tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c), v);
-    if (t < p.T) store_chunk<QF8, FAST>(row, n0 + c, v, d);
+      for (int col = hf * 128; col < hf * 128 + 128; col += 32) {
+        uint32_t v[32];
+        tmem_ld32(acc + static_cast<uint32_t>(col), v);
+        stage_chunk<QF8, FAST>(sC, r, col, v, d);
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bars.acc_empty[b])) : "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      bar_sync(2 + hf, 128);
+      if (issuer) {
+#pragma unroll
+        for (int sl = hf * (128 / kSlabCols); sl < (hf + 1) * (128 / kSlabCols); ++sl)
+          tma_store_3d(tmC, sC + static_cast<uint32_t>(sl) * kSlabC, c.nt * kN + sl * kSlabCols, c.h, c.m0);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+    }
+    if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  } else {
+    // rotary warps: the 64 pe values of 64 tokens of every tile
+    const int slot = static_cast<int>(threadIdx.x) - 32 * kPeWarp0;
+    pdl_wait();  // q_pe comes from the upstream kernel
+    for (int i = 0; i < count; ++i) {
+      const TileCoord c = tile_at(first + i, mt);
+      pe_part<QF8, ROPE, FAST>(p, c.m0, c.nt, c.h, slot, d);
+    }
   }
 }
 
 template <bool QF8, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
-    absorb_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
+    absorb_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmC, const Params p) {
   extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ __align__(8) Bars bars;
   __shared__ uint32_t tmem_slot;
-  __shared__ uint32_t fail;
+  __shared__ uint32_t abort_flag;
   const int warp = threadIdx.x >> 5;
   const uint32_t sbase = (smem_u32(dsmem) + 1023u) & ~1023u;
-  const uint32_t bar_tma = smem_u32(&bars[0]);
-  const uint32_t bar_mma = smem_u32(&bars[1]);
+  float q_scale = 1.0f;
+  if constexpr (QF8) q_scale = __ldg(p.q_scale);
 
-  Divisor d{};
-  d.fast = true;
-  if constexpr (QF8) d = make_divisor(__ldg(p.q_scale));
-
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (threadIdx.x == 0) {
-    fail = 0u;
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_tma) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma) : "memory");
+    abort_flag = 0u;
+    for (int st = 0; st < kStages; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars.a_full[st])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars.a_empty[st])) : "memory");
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars.b_full)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars.b_empty)) : "memory");
+    for (int b = 0; b < 2; ++b) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars.acc_full[b])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&bars.acc_empty[b])), "r"(kEpiWarps) : "memory");
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars.mma_done)) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -298,15 +541,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = tmem_slot;
 
+  Divisor d{};
+  d.fast = true;
+  if constexpr (QF8) d = make_divisor(q_scale);
   if (d.fast) {
-    tile<QF8, ROPE, true>(&tmA, &tmB, p, sbase, bar_tma, bar_mma, tmem, &fail, d);
+    run<QF8, ROPE, true>(&tmA, &tmB, &tmC, p, sbase, bars, tmem, &abort_flag, d);
   } else {
-    tile<QF8, ROPE, false>(&tmA, &tmB, p, sbase, bar_tma, bar_mma, tmem, &fail, d);
+    run<QF8, ROPE, false>(&tmA, &tmB, &tmC, p, sbase, bars, tmem, &abort_flag, d);
   }
 
+  // every MMA has completed (the MMA warp waited for its final commit) and
+  // every copy has landed (the TMA warp drained them): free the TMEM
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
@@ -389,6 +637,21 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
       return MLA_ERR_INVALID_ARG;
   }
 
+  // C: q_out as (column, h, t), box (one 128-byte column slab, 1, 128), written
+  // from the 128-byte swizzled staging tile; rows past T are not written
+  CUtensorMap tmC;
+  {
+    const cuuint64_t esz = qf8 ? 1 : 2;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kRow), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kRow) * esz, static_cast<cuuint64_t>(kRow * H) * esz};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), 1, static_cast<cuuint32_t>(kM)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(&tmC, qf8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q_out, dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_INVALID_ARG;
+  }
+
   Params prm;
   prm.q_pe = static_cast<const uint16_t*>(q_pe);
   prm.qp_st = qp_st;
@@ -401,6 +664,8 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
   prm.H = static_cast<int32_t>(H);
   prm.q_out = static_cast<uint8_t*>(q_out);
   prm.status = status;
+  prm.pe_vec = aligned(q_pe, 16) && (T == 1 || qp_st % 8 == 0) && (H == 1 || qp_sh % 8 == 0);
+  prm.tab_vec = rope && aligned(cos_sin, 16);
 
   const int k = (qf8 ? 2 : 0) | (rope ? 1 : 0);
   static const void* const kernels[4] = {kernel_for<false, false>(), kernel_for<false, true>(),
@@ -417,7 +682,13 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
   }
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(((T + kM - 1) / kM) * 2), static_cast<unsigned>(H), 1);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  const int64_t tiles = 2 * H * ((T + kM - 1) / kM);
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
@@ -428,7 +699,7 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  void* args[] = {&tmA, &tmB, &prm};
+  void* args[] = {&tmA, &tmB, &tmC, &prm};
   const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();

@@ -22,8 +22,8 @@ from mla_decode_attention_10_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _gpu(w, extra=0):
-    d = w.to("cuda")
+def _gpu(w, extra=0, d=None):
+    d = w.to("cuda") if d is None else d
     q = torch.full((w.T, w.H, 576), 0x7F if w.q_fp8 else 0, dtype=torch.uint8 if w.q_fp8 else torch.bfloat16,
                    device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -108,3 +108,46 @@ def test_absorbed_rows_behind_producer_with_pdl():
     assert rc == E.MLA_OK
     torch.cuda.synchronize()
     _check(w, q.cpu(), 0)
+
+
+@pytest.mark.parametrize("flags", [W.FLAG_ROPE, W.FLAG_ROPE | W.FLAG_Q_FP8])
+def test_absorbed_rows_positions_out_of_range(flags):
+    """Positions outside the table leave those tokens' pe values unrotated and
+    set the status bit; 37 tokens leave a ragged last group of rows."""
+    w = W.make_absorb("oor", 37, 3, flags, seed=11, rope_rows=64, scale=0.05)
+    w.positions[::5] = -1
+    w.positions[3::7] = 64
+    q, st = _gpu(w)
+    assert st == E.MLA_STATUS_POS_RANGE
+    _check(w, q, st)
+
+
+@pytest.mark.parametrize("layout", ["pe_offset", "table_offset", "pe_stride_68", "pe_stride_72"])
+def test_absorbed_rows_unaligned_pe_and_table(layout):
+    """q_pe or the cos/sin table off the 16-byte grid (2- or 4-byte aligned,
+    or a row stride that is not a multiple of 8 elements) take the scalar
+    load path; a stride of 72 keeps the vector path on a strided view."""
+    w = W.make_absorb("ua", 70, 3, W.FLAG_ROPE | W.FLAG_Q_FP8, seed=21, rope_rows=256, scale=0.05)
+    d = w.to("cuda")
+    if layout == "pe_offset":
+        buf = torch.empty(w.T * w.H * 64 + 1, dtype=torch.bfloat16, device="cuda")
+        buf[1:].copy_(d.q_pe.reshape(-1))
+        d.q_pe = buf[1:].view(w.T, w.H, 64)
+    elif layout == "table_offset":
+        buf = torch.empty(d.cos_sin.numel() + 1, dtype=torch.float32, device="cuda")
+        buf[1:].copy_(d.cos_sin.reshape(-1))
+        d.cos_sin = buf[1:].view(d.cos_sin.shape)
+    else:
+        width = int(layout.rsplit("_", 1)[1])
+        buf = torch.zeros(w.T, w.H, width, dtype=torch.bfloat16, device="cuda")
+        buf[:, :, :64].copy_(d.q_pe)
+        d.q_pe = buf[:, :, :64]
+    q, st = _gpu(w, d=d)
+    _check(w, q, st)
+    w_bf16 = W.make_absorb("ua16", 70, 3, W.FLAG_ROPE, seed=22, rope_rows=256)
+    d16 = w_bf16.to("cuda")
+    buf = torch.empty(w_bf16.T * w_bf16.H * 64 + 1, dtype=torch.bfloat16, device="cuda")
+    buf[1:].copy_(d16.q_pe.reshape(-1))
+    d16.q_pe = buf[1:].view(w_bf16.T, w_bf16.H, 64)
+    q, st = _gpu(w_bf16, d=d16)
+    _check(w_bf16, q, st)
