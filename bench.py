@@ -478,6 +478,7 @@ def run_ours(args, rank, world, local_rank):
         line["context_errors"] = context_errors
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args.workload)
+        line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(args.workload)
     return line
 
 
@@ -751,6 +752,29 @@ def cpu_baseline(name: str, seconds: float = 10.0):
     return {"value": round(dt / n * 1e6, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} calls of {name} (T={w.T}, H={w.H}) in {dt:.1f} s, one host thread "
                       f"({os.cpu_count()} cores on the host)"}
+
+
+def cpu_baseline_all_cores(name: str, seconds: float = 5.0):
+    """The same oracle function, as it stands, on contiguous token slices on
+    every host core at once (one std::thread per slice inside the oracle
+    library).  Reported as a baseline only."""
+    import oracle
+    w = named_variant(name, 0)
+    cores = max(1, min(os.cpu_count() or 1, w.T))
+
+    def call():
+        oracle.run(w.q_nope, w.q_pe, w.kv_c, w.k_pe, w.slot_mapping, w.cache, w.flags, positions=w.positions,
+                   cos_sin=w.cos_sin, q_scale=w.q_scale, kv_scale=w.kv_scale, threads=cores)
+
+    call()
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        call()
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(dt / n * 1e6, 2), "unit": UNIT, "cores": cores, "kind": "oracle, token slices on threads",
+            "sample": f"{n} calls of {name} (T={w.T}, H={w.H}) in {dt:.1f} s, {cores} threads of "
+                      f"{-(-w.T // cores)} tokens at most; baseline only"}
 
 
 def run_reference(args, rank, world):

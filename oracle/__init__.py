@@ -40,6 +40,8 @@ def lib() -> ctypes.CDLL:
         L.mla_oracle_run.argtypes = [vp, i64, i64, vp, i64, i64, vp, i64, vp, i64,
                                      vp, vp, vp, i64, vp, vp,
                                      i64, i64, i64, i64, u32, vp, vp, vp]
+        L.mla_oracle_run_threads.restype = ctypes.c_int
+        L.mla_oracle_run_threads.argtypes = L.mla_oracle_run.argtypes + [ctypes.c_int]
         L.mla_oracle_absorb_run.restype = ctypes.c_int
         L.mla_oracle_absorb_run.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, vp,
                                             i64, i64, u32, vp, vp]
@@ -69,12 +71,14 @@ def run(q_nope: torch.Tensor, q_pe: torch.Tensor, kv_c: torch.Tensor, k_pe: torc
         slot_mapping: torch.Tensor, cache: torch.Tensor, flags: int,
         positions: Optional[torch.Tensor] = None, cos_sin: Optional[torch.Tensor] = None,
         q_scale: Optional[torch.Tensor] = None, kv_scale: Optional[torch.Tensor] = None,
-        ) -> Tuple[torch.Tensor, int]:
+        threads: int = 1) -> Tuple[torch.Tensor, int]:
     """Run the oracle on host tensors.
 
     ``cache`` ([num_blocks, block_size, 576], bf16 or uint8 for e4m3 bytes) is
     updated in place.  Returns ``(q_out, status)`` where ``q_out`` is
     [T, H, 576] bf16, or uint8 e4m3 bytes when ``FLAG_Q_FP8`` is set.
+    ``threads`` > 1 runs the same function on that many contiguous token
+    slices at once (the benchmark's all-cores baseline; slots must be unique).
     """
     T, H = q_nope.shape[0], q_nope.shape[1]
     assert q_nope.dtype == torch.bfloat16 and q_pe.dtype == torch.bfloat16
@@ -89,7 +93,9 @@ def run(q_nope: torch.Tensor, q_pe: torch.Tensor, kv_c: torch.Tensor, k_pe: torc
     q_fp8 = bool(flags & FLAG_Q_FP8)
     q_out = torch.empty((T, H, ROW), dtype=torch.uint8 if q_fp8 else torch.bfloat16)
     status = ctypes.c_int32(0)
-    rc = lib().mla_oracle_run(
+    fn = lib().mla_oracle_run if threads <= 1 else lib().mla_oracle_run_threads
+    extra = () if threads <= 1 else (int(threads),)
+    rc = fn(
         _ptr(q_nope), q_nope.stride(0), q_nope.stride(1),
         _ptr(q_pe), q_pe.stride(0), q_pe.stride(1),
         _ptr(kv_c), kv_c.stride(0),
@@ -98,7 +104,7 @@ def run(q_nope: torch.Tensor, q_pe: torch.Tensor, kv_c: torch.Tensor, k_pe: torc
         _ptr(positions), _ptr(cos_sin), cos_sin.shape[0] if cos_sin is not None else 0,
         _ptr(q_scale), _ptr(kv_scale),
         T, H, cache.shape[1], cache.shape[0], flags,
-        _ptr(q_out), _ptr(cache), ctypes.addressof(status))
+        _ptr(q_out), _ptr(cache), ctypes.addressof(status), *extra)
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return q_out, status.value

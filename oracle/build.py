@@ -22,7 +22,7 @@ def build(force: bool = False) -> str:
             and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
         return LIB
     cmd = ["g++", "-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math",
-           "-fno-finite-math-only", "-Wall", "-Wextra", "-shared", "-fPIC",
+           "-fno-finite-math-only", "-Wall", "-Wextra", "-shared", "-fPIC", "-pthread",
            SRC, "-o", LIB + ".tmp"]
     subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)

@@ -1,6 +1,8 @@
 // mla_oracle.cpp -- TEST INFRASTRUCTURE ONLY.
 //
-// A plain, slow, single-threaded CPU oracle of the fused MLA decode epilogue:
+// A plain, slow, single-threaded CPU oracle of the fused MLA decode epilogue
+// (mla_oracle_run_threads only runs that same function on token slices in
+// parallel, for the benchmark's all-cores baseline):
 // per token it builds H latent query rows and one latent KV-cache row, each
 // 576 wide, exactly as the operation is defined, with no blocking, fusion or
 // reordering.  Only the tests, the smoke check and the benchmark's CPU
@@ -35,6 +37,8 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <thread>
+#include <vector>
 
 namespace {
 
@@ -297,6 +301,47 @@ int mla_oracle_absorb_run(const uint16_t* q_nope_c, int64_t qc_st, int64_t qc_sh
   }
   if (status != nullptr) *status |= st;
   return 0;
+}
+
+// The benchmark's all-cores baseline: mla_oracle_run, unchanged, on
+// `threads` contiguous token slices at once (one std::thread each).  Tokens
+// are independent and the caller's slots are unique, so the slices write
+// disjoint rows; nothing is reordered inside a slice.
+int mla_oracle_run_threads(const uint16_t* q_nope, int64_t qn_st, int64_t qn_sh,
+                           const uint16_t* q_pe, int64_t qp_st, int64_t qp_sh,
+                           const uint16_t* kv_c, int64_t kv_st,
+                           const uint16_t* k_pe, int64_t kp_st,
+                           const int64_t* slot_mapping, const int32_t* positions,
+                           const float* cos_sin, int64_t rope_rows,
+                           const float* q_scale, const float* kv_scale,
+                           int64_t T, int64_t H, int64_t block_size, int64_t num_blocks,
+                           uint32_t flags, void* q_out, void* cache, int32_t* status, int threads) {
+  if (threads < 1 || T < 0 || H < 1) return 1;
+  if (T == 0) return mla_oracle_run(q_nope, qn_st, qn_sh, q_pe, qp_st, qp_sh, kv_c, kv_st, k_pe, kp_st, slot_mapping,
+                                    positions, cos_sin, rope_rows, q_scale, kv_scale, T, H, block_size, num_blocks,
+                                    flags, q_out, cache, status);
+  const int n = static_cast<int>(threads < T ? threads : T);
+  const int64_t q_row_bytes = (flags & kFlagQFp8) ? kRow : 2 * kRow;
+  std::vector<int32_t> st(n, 0);
+  std::vector<int> rc(n, 0);
+  std::vector<std::thread> pool;
+  for (int i = 0; i < n; ++i) {
+    const int64_t t0 = T * i / n, t1 = T * (i + 1) / n;
+    pool.emplace_back([=, &st, &rc]() {
+      rc[i] = mla_oracle_run(q_nope + t0 * qn_st, qn_st, qn_sh, q_pe + t0 * qp_st, qp_st, qp_sh, kv_c + t0 * kv_st,
+                             kv_st, k_pe + t0 * kp_st, kp_st, slot_mapping + t0,
+                             positions != nullptr ? positions + t0 : nullptr, cos_sin, rope_rows, q_scale, kv_scale,
+                             t1 - t0, H, block_size, num_blocks, flags,
+                             static_cast<uint8_t*>(q_out) + t0 * H * q_row_bytes, cache, &st[i]);
+    });
+  }
+  int result = 0;
+  for (int i = 0; i < n; ++i) {
+    pool[i].join();
+    if (rc[i] != 0) result = rc[i];
+    if (status != nullptr) *status |= st[i];
+  }
+  return result;
 }
 
 }  // extern "C"

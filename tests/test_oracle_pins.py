@@ -416,3 +416,21 @@ def test_brute_force_tiny_all_flags(flags, T):
         assert torch.equal(rows, ekv)
     else:
         assert torch.equal(_bits16(rows), _bits16(ekv))
+
+
+@pytest.mark.parametrize("flags", [0, W.FLAG_ROPE, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8])
+@pytest.mark.parametrize("threads", [2, 3, 64])
+def test_threaded_driver_equals_single_thread(flags, threads):
+    """The all-cores baseline runs the same per-token function on token
+    slices: results and status bits equal the single-threaded run."""
+    w = W.make("thr", 37, 5, flags, seed=41, num_blocks=4, block_size=16)
+    cache1, cache2 = w.cache.clone(), w.cache.clone()
+    if flags & W.FLAG_ROPE:
+        w.positions[::9] = -3  # a status bit from some slices
+    q1, s1 = oracle.run(w.q_nope, w.q_pe, w.kv_c, w.k_pe, w.slot_mapping, cache1, flags, positions=w.positions,
+                        cos_sin=w.cos_sin, q_scale=w.q_scale, kv_scale=w.kv_scale)
+    q2, s2 = oracle.run(w.q_nope, w.q_pe, w.kv_c, w.k_pe, w.slot_mapping, cache2, flags, positions=w.positions,
+                        cos_sin=w.cos_sin, q_scale=w.q_scale, kv_scale=w.kv_scale, threads=threads)
+    assert s1 == s2
+    assert torch.equal(q1.view(torch.uint8), q2.view(torch.uint8))
+    assert torch.equal(cache1.view(torch.uint8), cache2.view(torch.uint8))
