@@ -151,3 +151,12 @@ def test_absorbed_rows_unaligned_pe_and_table(layout):
     d16.q_pe = buf[1:].view(w_bf16.T, w_bf16.H, 64)
     q, st = _gpu(w_bf16, d=d16)
     _check(w_bf16, q, st)
+
+
+def test_absorbed_rows_many_heads_reload_weights():
+    """T=100, H=200: 400 one-tile (head, column half) groups over at most 148
+    persistent CTAs, so a CTA loads new weights for two or three successive
+    groups (the weight buffer's empty/full phases alternate)."""
+    w = W.make_absorb("heads", 100, 200, W.FLAG_ROPE | W.FLAG_Q_FP8, seed=17, rope_rows=4096, scale=0.05)
+    q, st = _gpu(w)
+    _check(w, q, st)
