@@ -228,3 +228,43 @@ def test_absorb_validation(lib, kw, code):
     args.update(T=0, q_nope_c=None, w_uk=None, q_out=None)
     if code != E.MLA_ERR_UNSUPPORTED and kw.get("H", 1) >= 1 and kw.get("H", 1) < 65536 and kw.get("T", 0) >= 0:
         assert E.mla_absorb_launch(**args) == E.MLA_OK
+
+
+C_USER = r"""
+#include "mla_epilogue.h"
+#include "mla_absorb.h"
+#include "mla_harness.h"
+#include <stdio.h>
+#include <string.h>
+
+int main(void) {
+  mla_plan plan;
+  if (mla_epilogue_plan(64, 16, MLA_FLAG_ROPE, 148, &plan) != MLA_OK) return 1;
+  /* T == 0: nothing to read or write, no CUDA call */
+  if (mla_epilogue_launch(NULL, 0, 0, NULL, 0, 0, NULL, 0, NULL, 0, NULL, NULL, NULL, 0, NULL, NULL,
+                          0, 16, 64, 1, 0, NULL, NULL, NULL, NULL) != MLA_OK) return 2;
+  if (mla_absorb_launch(NULL, 0, 0, NULL, NULL, 0, 0, NULL, NULL, 0, NULL, 0, 1, 0, NULL, NULL, NULL) != MLA_OK) return 3;
+  /* a bad argument is refused on the host */
+  if (mla_absorb_launch(NULL, 0, 0, NULL, NULL, 0, 0, NULL, NULL, 0, NULL, 4, 0, 0, NULL, NULL, NULL)
+      != MLA_ERR_INVALID_ARG) return 4;
+  if (strlen(mla_status_string(MLA_ERR_ALIGNMENT)) == 0) return 5;
+  printf("%d %lld\n", (int)plan.mode, (long long)plan.blocks);
+  return 0;
+}
+"""
+
+
+def test_headers_are_plain_c_and_link(lib, tmp_path):
+    """A C11 program (no C++, no CUDA headers) includes every header, links
+    the library and calls its host-side paths."""
+    src = tmp_path / "use.c"
+    src.write_text(C_USER)
+    exe = tmp_path / "use"
+    libdir = os.path.dirname(B.LIB)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-l:" + os.path.basename(B.LIB), "-o", str(exe)], check=True)
+    env = dict(os.environ, LD_LIBRARY_PATH=libdir + os.pathsep + os.environ.get("LD_LIBRARY_PATH", ""))
+    out = subprocess.run([str(exe)], env=env, capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
+    mode, blocks = out.stdout.split()
+    assert int(mode) == E.MLA_MODE_SPLIT and int(blocks) > 0
