@@ -674,10 +674,19 @@ def absorb_measure(E, stream, device, peak_gbs):
 def run_e2e(args, w0, stream, device, world):
     """Same metric through the user-facing call, with host buffers: every step
     copies its inputs from pinned host memory, runs the epilogue and copies
-    q_out back, all on one stream, timed with CUDA events.  The per-step
-    inputs (q_nope, q_pe, kv_c, k_pe, slot_mapping, positions) sit in one
-    pinned staging buffer at 16-byte aligned offsets, so each step is one
-    host-to-device copy, the call, and one device-to-host copy."""
+    q_out back, timed with CUDA events.  The per-step inputs (q_nope, q_pe,
+    kv_c, k_pe, slot_mapping, positions) sit in one pinned staging buffer at
+    16-byte aligned offsets, so each step is one host-to-device copy, the
+    call, and one device-to-host copy.
+
+    Three schedules are timed.  Serial: all three on the launch stream, one
+    step after the other.  Pipelined: uploads, calls and downloads on three
+    streams with two buffer sets, the way a serving loop overlaps them: step
+    i+1's upload runs while step i computes and step i-1's result comes back;
+    events order every reuse of a buffer.  Graphed (the reported value): the
+    pipelined schedule of 20 steps captured once as a CUDA graph, with its
+    copy nodes, and replayed, as decode loops launch their steps; every
+    replayed step still moves its inputs and its result over the host link."""
     from mla_decode_attention_10_b200 import epilogue as E
     parts = [(k, getattr(w0, k).contiguous()) for k in ("q_nope", "q_pe", "kv_c", "k_pe", "slot_mapping", "positions")
              if getattr(w0, k) is not None]
@@ -685,48 +694,129 @@ def run_e2e(args, w0, stream, device, world):
     for k, v in parts:
         offsets[k] = total
         total += -(-v.numel() * v.element_size() // 16) * 16
-    host = torch.empty(total, dtype=torch.uint8).pin_memory()
-    for k, v in parts:
-        n = v.numel() * v.element_size()
-        host[offsets[k]:offsets[k] + n].copy_(v.view(-1).view(torch.uint8))
-    dbuf = torch.empty(total, dtype=torch.uint8, device=device)
-    dev = {k: dbuf[offsets[k]:offsets[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
-           for k, v in parts}
     cache = w0.cache.to(device)
     cos_sin = w0.cos_sin.to(device) if w0.cos_sin is not None else None
     qs = w0.q_scale.to(device) if w0.q_scale is not None else None
     ks = w0.kv_scale.to(device) if w0.kv_scale is not None else None
-    q_out = torch.empty((w0.T, w0.H, W.ROW), dtype=w0.q_out_dtype(), device=device)
-    q_host = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for _, v in parts)
-    d2h = q_host.numel() * q_host.element_size()
 
-    def step():
+    def buffer_set():
+        host = torch.empty(total, dtype=torch.uint8).pin_memory()
+        for k, v in parts:
+            n = v.numel() * v.element_size()
+            host[offsets[k]:offsets[k] + n].copy_(v.view(-1).view(torch.uint8))
+        dbuf = torch.empty(total, dtype=torch.uint8, device=device)
+        dev = {k: dbuf[offsets[k]:offsets[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+               for k, v in parts}
+        q_out = torch.empty((w0.T, w0.H, W.ROW), dtype=w0.q_out_dtype(), device=device)
+        q_host = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
+        return {"host": host, "dbuf": dbuf, "dev": dev, "q_out": q_out, "q_host": q_host}
+
+    sets = [buffer_set(), buffer_set()]
+    h2d = sum(v.numel() * v.element_size() for _, v in parts)
+    d2h = sets[0]["q_host"].numel() * sets[0]["q_host"].element_size()
+
+    def call(b, s):
+        dev = b["dev"]
+        E.fused_mla_decode_q_concat_kv_cache_insert(
+            dev["q_nope"], dev["q_pe"], dev["kv_c"], dev["k_pe"], cache, dev["slot_mapping"],
+            positions=dev.get("positions"), cos_sin=cos_sin, q_scale=qs, kv_scale=ks, q_out=b["q_out"], stream=s)
+
+    def serial_step():
+        b = sets[0]
         with torch.cuda.stream(stream):
-            dbuf.copy_(host, non_blocking=True)
-            E.fused_mla_decode_q_concat_kv_cache_insert(
-                dev["q_nope"], dev["q_pe"], dev["kv_c"], dev["k_pe"], cache, dev["slot_mapping"],
-                positions=dev.get("positions"), cos_sin=cos_sin, q_scale=qs, kv_scale=ks,
-                q_out=q_out, stream=stream)
-            q_host.copy_(q_out, non_blocking=True)
+            b["dbuf"].copy_(b["host"], non_blocking=True)
+            call(b, stream)
+            b["q_host"].copy_(b["q_out"], non_blocking=True)
+
+    up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+    ev = [{n: torch.cuda.Event() for n in ("up", "comp", "down")} for _ in sets]
+    for e in ev:  # every event starts out recorded, so the first waits pass
+        for n in e:
+            e[n].record(stream)
+
+    def pipelined_step(i, first=False):
+        b, e = sets[i % 2], ev[i % 2]
+        if not first:
+            up.wait_event(e["comp"])   # the call two steps back has read this input buffer
+        with torch.cuda.stream(up):
+            b["dbuf"].copy_(b["host"], non_blocking=True)
+        e["up"].record(up)
+        stream.wait_event(e["up"])
+        if not first:
+            stream.wait_event(e["down"])  # the download two steps back has read this q_out
+        call(b, stream)
+        e["comp"].record(stream)
+        down.wait_event(e["comp"])
+        with torch.cuda.stream(down):
+            b["q_host"].copy_(b["q_out"], non_blocking=True)
+        e["down"].record(down)
+
+    def timed_run(step_fn, k):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier(device)
+        e0.record(stream)
+        up.wait_stream(stream)
+        down.wait_stream(stream)
+        for i in range(k):
+            step_fn(i)
+        stream.wait_stream(up)
+        stream.wait_stream(down)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(device)
+        return max_over_ranks(e0.elapsed_time(e1), device)
 
     k = max(10, min(args.steps, 200))
     for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    barrier(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(k):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(device)
-    ms = max_over_ranks(e0.elapsed_time(e1), device)
-    return {"value": round(job_us_per_call(ms, k, world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": k,
-            "path": "epilogue.fused_mla_decode_q_concat_kv_cache_insert; inputs from one pinned staging buffer "
-                    "(one host-to-device copy), q_out back to pinned host memory, all on the launch stream"}
+        serial_step()
+    serial_ms = timed_run(lambda i: serial_step(), k)
+    for i in range(max(args.warmup, 3)):
+        pipelined_step(i)
+    pipe_ms = timed_run(pipelined_step, k)
+    # the same schedule as one CUDA graph of G steps (the first two steps of
+    # a replay wait for nothing: the previous replay has completed)
+    G = 20
+    graph_ms, graph_note = None, None
+    try:
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            up.wait_stream(stream)
+            down.wait_stream(stream)
+            for i in range(G):
+                pipelined_step(i, first=i < 2)
+            stream.wait_stream(up)
+            stream.wait_stream(down)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                g.replay()
+        reps = max(1, k // G)
+
+        def replay(i):
+            with torch.cuda.stream(stream):
+                g.replay()
+
+        graph_ms = timed_run(replay, reps)
+        graph_steps = G * reps
+    except RuntimeError as exc:  # capture refused: report the stream-pipelined figure
+        graph_note = f"graph capture failed: {exc}"[:200]
+    if graph_ms is not None:
+        value = job_us_per_call(graph_ms, graph_steps, world)
+    else:
+        value = job_us_per_call(pipe_ms, k, world)
+    out = {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": graph_steps if graph_ms is not None else k,
+            "pipelined_value": round(job_us_per_call(pipe_ms, k, world), 3),
+            "serial_value": round(job_us_per_call(serial_ms, k, world), 3),
+            "path": "epilogue.fused_mla_decode_q_concat_kv_cache_insert; per step one host-to-device copy of the "
+                    "inputs from a pinned staging buffer, the call, and q_out back to pinned host memory; value: "
+                    "the pipelined schedule (uploads, calls, downloads on three streams, two buffer sets) captured "
+                    "as a CUDA graph of 20 steps and replayed; pipelined_value: the same schedule issued step by "
+                    "step; serial_value: all on the launch stream, one step after the other"}
+    if graph_note:
+        out["note"] = graph_note
+    return out
 
 
 # ---------------------------------------------------------------------------------------
