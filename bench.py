@@ -777,7 +777,7 @@ def run_e2e(args, w0, stream, device, world):
     # the same schedule as one CUDA graph of G steps (the first two steps of
     # a replay wait for nothing: the previous replay has completed)
     G = 20
-    graph_ms, graph_note = None, None
+    graph_ms, graph_note, g = None, None, None
     try:
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -791,6 +791,12 @@ def run_e2e(args, w0, stream, device, world):
         with torch.cuda.stream(stream):
             for _ in range(2):
                 g.replay()
+        torch.cuda.synchronize()
+    except RuntimeError as exc:  # capture refused: report the stream-pipelined figure
+        graph_note = f"graph capture failed: {exc}"[:200]
+        g = None
+    # every rank takes the same branch, so the collectives inside timed_run match
+    if max_over_ranks(0.0 if g is not None else 1.0, device) == 0.0:
         reps = max(1, k // G)
 
         def replay(i):
@@ -799,8 +805,8 @@ def run_e2e(args, w0, stream, device, world):
 
         graph_ms = timed_run(replay, reps)
         graph_steps = G * reps
-    except RuntimeError as exc:  # capture refused: report the stream-pipelined figure
-        graph_note = f"graph capture failed: {exc}"[:200]
+    elif graph_note is None:
+        graph_note = "graph capture failed on another rank"
     if graph_ms is not None:
         value = job_us_per_call(graph_ms, graph_steps, world)
     else:
