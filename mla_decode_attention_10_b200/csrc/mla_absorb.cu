@@ -18,8 +18,11 @@
 //     128-byte swizzle, frees the accumulator, and one thread per half sends
 //     each 128-byte column slab out with one bulk tensor store, so HBM sees
 //     whole-line writes;
-//   * warps 10..13 (rotary): per tile, the 64 pe values of 64 of its tokens,
-//     two threads per token, every load issued before any is used.
+//   * warps 10..13 (rotary): the 64 pe values of every head of the CTA's
+//     share of the tokens, two threads per (token, head), every load issued
+//     before any is used; consecutive threads take consecutive heads of one
+//     token, so a token's table row is read once per warp and its q_pe rows
+//     as one contiguous run.
 // The loads of tile i+1, its MMAs and the epilogue of tile i overlap.  Every
 // wait is bounded: on timeout the kernel sets a status bit, every role stops,
 // the copies in flight are waited for (bounded), TMEM is freed and the kernel
@@ -194,12 +197,12 @@ __device__ __forceinline__ void stage_chunk(uint32_t sC, int r, int col, const u
   }
 }
 
-// The 64 rotary values of 64 of a tile's tokens: the tile of column half nt
-// covers tokens m0 + 64 nt .. m0 + 64 nt + 63, two threads (tid 2j, 2j+1)
-// per token, each 16 of the 32 rotation pairs (i, i+32).  Every thread
-// issues all of its loads (its q_pe values and its cos and sin entries, as
-// 16-byte vectors when the host found them aligned) before it uses any, so
-// a tile costs about two memory round trips (position, then table).
+// The 64 rotary values of one (token, head) row, half of them: token
+// m0 + 64 nt + tid / 2, rotation pairs (i, i+32) for i in 16 (tid & 1) ..
+// 16 (tid & 1) + 15.  The thread issues all of its loads (its q_pe values and
+// its cos and sin entries, as 16-byte vectors when the host found them
+// aligned) before it uses any: about two memory round trips (position, then
+// table).
 template <bool QF8, bool ROPE, bool FAST>
 __device__ __forceinline__ void pe_part(const Params& p, int m0, int nt, int h, int tid, const Divisor& d) {
   const int t = m0 + 64 * nt + (tid >> 1);
@@ -492,12 +495,19 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
     }
     if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   } else {
-    // rotary warps: the 64 pe values of 64 tokens of every tile
+    // rotary warps: the 64 pe values of every head of this CTA's share of
+    // the tokens (independent of its tiles), item (t, h, half) per thread,
+    // consecutive threads on consecutive heads of one token
     const int slot = static_cast<int>(threadIdx.x) - 32 * kPeWarp0;
+    const int64_t tb0 = static_cast<int64_t>(p.T) * bx / static_cast<int>(gridDim.x);
+    const int64_t tb1 = static_cast<int64_t>(p.T) * (bx + 1) / static_cast<int>(gridDim.x);
+    const int64_t per_token = 2 * static_cast<int64_t>(p.H);
+    const int64_t items = (tb1 - tb0) * per_token;
     pdl_wait();  // q_pe comes from the upstream kernel
-    for (int i = 0; i < count; ++i) {
-      const TileCoord c = tile_at(first + i, mt);
-      pe_part<QF8, ROPE, FAST>(p, c.m0, c.nt, c.h, slot, d);
+    for (int64_t it = slot; it < items; it += 32 * kPeWarps) {
+      const int64_t tt = it / per_token;
+      const int rem = static_cast<int>(it - tt * per_token);
+      pe_part<QF8, ROPE, FAST>(p, static_cast<int>(tb0 + tt), 0, rem >> 1, rem & 1, d);
     }
   }
 }
