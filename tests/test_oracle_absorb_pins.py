@@ -33,6 +33,66 @@ def test_identity_weights_copy_the_input():
     assert torch.equal(_bits(q[..., 512:]), _bits(w.q_pe))
 
 
+def test_permutation_weights_select_one_input_each():
+    """W_UK[h, j, k] = 1 exactly when k = (5 j + 3 h) mod 128: latent value j
+    of head h is input element (5 j + 3 h) mod 128 of the same token and
+    head, bit for bit.  The map differs per head and is not symmetric in
+    (j, k), so a transposed weight index, a wrong head or a wrong token
+    fails."""
+    T, H = 4, 3
+    w = W.make_absorb("perm", T, H, 0, seed=2, q_nope_row=136)
+    w.w_uk.zero_()
+    for h in range(H):
+        for j in range(512):
+            w.w_uk[h, j, (5 * j + 3 * h) % 128] = 1.0
+    q, st = _run(w)
+    assert st == 0
+    src = w.q_nope_c.contiguous()
+    for h in range(H):
+        idx = torch.tensor([(5 * j + 3 * h) % 128 for j in range(512)])
+        assert torch.equal(_bits(q[:, h, :512]), _bits(src[:, h, idx]))
+
+
+def test_one_hot_queries_read_one_weight_column():
+    """q_nope_c[t, h] = e_k with k = (7 t + h) mod 128: latent value j is
+    W_UK[h, j, k], bit for bit (one exact product, one term)."""
+    T, H = 3, 2
+    w = W.make_absorb("onehot", T, H, 0, seed=4)
+    w.q_nope_c.zero_()
+    for t in range(T):
+        for h in range(H):
+            w.q_nope_c[t, h, (7 * t + h) % 128] = 1.0
+    q, st = _run(w)
+    assert st == 0
+    for t in range(T):
+        for h in range(H):
+            assert torch.equal(_bits(q[t, h, :512]), _bits(w.w_uk[h, :, (7 * t + h) % 128]))
+
+
+def test_exact_sums_cancellation_and_ties():
+    """Sums whose exact value is known: 2^24 + 1 - 2^24 = 1 (lost by fp32
+    accumulation in that order); 1 + 2^-9 + 2^-9 = 1 + 2^-8, a bf16 tie
+    that rounds to even (1.0); 1 + 2^-9 + 2^-9 + 2^-20, just above the tie
+    (1 + 2^-7).  The latent values are rounded once, from the exact sum."""
+    w = W.make_absorb("sums", 1, 1, 0, seed=6)
+    w.q_nope_c.zero_()
+    w.w_uk.zero_()
+    q_vals = {0: 2.0 ** 24, 1: 1.0, 2: -(2.0 ** 24), 3: 1.0, 4: 2.0 ** -9, 5: 2.0 ** -9, 6: 2.0 ** -20}
+    for k, v in q_vals.items():
+        w.q_nope_c[0, 0, k] = v
+    for k in (0, 1, 2):
+        w.w_uk[0, 0, k] = 1.0          # latent 0: cancellation
+    for k in (3, 4, 5):
+        w.w_uk[0, 1, k] = 1.0          # latent 1: exactly on the tie
+    for k in (3, 4, 5, 6):
+        w.w_uk[0, 2, k] = 1.0          # latent 2: just above it
+    q, st = _run(w)
+    assert st == 0
+    got = q[0, 0, :3].float().tolist()
+    assert got == [1.0, 1.0, 1.0 + 2.0 ** -7], got
+    assert torch.all(q[0, 0, 3:512].float() == 0)
+
+
 @pytest.mark.parametrize("flags", [0, W.FLAG_Q_FP8])
 def test_small_integer_products_match_numpy(flags):
     """Inputs that are small integers times 2^-3 make every sum exact in
