@@ -434,3 +434,24 @@ def test_threaded_driver_equals_single_thread(flags, threads):
     assert s1 == s2
     assert torch.equal(q1.view(torch.uint8), q2.view(torch.uint8))
     assert torch.equal(cache1.view(torch.uint8), cache2.view(torch.uint8))
+
+
+def test_query_and_cache_rows_use_their_own_scale():
+    """q_scale 0.5, kv_scale 2.0, constant inputs: every query byte is the
+    e4m3 code of 1 / 0.5 = 2 (0x40) and every cache byte that of 2 / 2 = 1
+    (0x38), from the format's definition (bias 7, three mantissa bits).
+    Swapping the two scales, or using one for both, changes one of them."""
+    w = W.make("scales", 3, 2, W.FLAG_Q_FP8 | W.FLAG_KV_FP8, seed=8, num_blocks=1, block_size=16)
+    w.q_nope.fill_(1.0)
+    w.q_pe.fill_(1.0)
+    w.kv_c.fill_(2.0)
+    w.k_pe.fill_(2.0)
+    w.q_scale = torch.tensor([0.5], dtype=torch.float32)
+    w.kv_scale = torch.tensor([2.0], dtype=torch.float32)
+    cache = w.cache.clone()
+    q, st = oracle.run(w.q_nope, w.q_pe, w.kv_c, w.k_pe, w.slot_mapping, cache, w.flags,
+                       q_scale=w.q_scale, kv_scale=w.kv_scale)
+    assert st == 0
+    assert torch.all(q == 0x40)
+    rows = cache.view(-1, 576)[w.slot_mapping]
+    assert torch.all(rows == 0x38)
