@@ -268,3 +268,16 @@ def test_headers_are_plain_c_and_link(lib, tmp_path):
     assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
     mode, blocks = out.stdout.split()
     assert int(mode) == E.MLA_MODE_SPLIT and int(blocks) > 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No silent fallback: with the library absent, the binding raises before
+    any work is done, and the torch-level call does too."""
+    monkeypatch.setattr(E, "_lib", None)
+    monkeypatch.setattr(E, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="no CPU or PyTorch fallback"):
+        E.lib()
+    with pytest.raises(RuntimeError):
+        E.status_string(0)
+    with pytest.raises(RuntimeError):
+        E.mla_epilogue_launch(0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 1, 1, 64, 1, 0, 0, 0, 0, 0)
