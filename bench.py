@@ -4,21 +4,26 @@
                     [--workload NAME] [--no-sweep] [--no-cpu-baseline]
 
 One step is one call of the epilogue (the whole hot path) on one batch of
-the workload.  Default workload: the row-split boundary case, T=64 tokens,
-H=16 heads, bf16, RoPE (the decode size at which the vLLM PR #54896 report
-switches to three warps per row).  Inputs are device-resident when the timed
-region starts; consecutive steps rotate over input sets whose total is more
-than twice the L2, so every step reads HBM.  The K calls are replayed from
-CUDA graphs on one stream and timed with CUDA events on that stream; the
-bare-launch floor is an empty kernel with the same grid, block and launch
-attributes, timed the same way.
+the workload.  Default workload: the large batch, T=8192 tokens, H=16 heads,
+RoPE and e4m3 query and cache rows, the one configuration with T >= 4096
+(where the bandwidth target applies) and the largest that fits one GPU.
+Inputs are device-resident when a timed region starts; consecutive calls
+rotate over input sets whose total is more than twice the L2, and L2 is
+written over before every timed region, so every call reads HBM.  The K
+calls are replayed from CUDA graphs on one stream, timed with CUDA events on
+that stream; the K-call region is timed REPLAYS times and the median is
+reported.  The bare-launch floor is an empty kernel with the same grid,
+block and launch attributes, timed the same way.
 
 Printed: one JSON line (rank 0) with the metric in microseconds per call,
-achieved HBM GB/s against the measured copy bandwidth, the launch floor, a
-sweep over the other workload sizes, the end-to-end time through the Python
-API with pinned host buffers, the CPU oracle as a baseline and the SM clocks
-seen under load.  ``--impl reference`` times the CPU oracle instead (the only
-reference implementation this operation has here).
+achieved HBM GB/s against the measured copy bandwidth, the launch floor, the
+decode sizes T = 1 .. 64 standalone and behind the synthetic producer with
+programmatic dependent launch (against an empty dependent kernel), the
+launch-to-end latency of isolated calls, a sweep over the other workload
+sizes, the end-to-end time through the Python API with pinned host buffers,
+the CPU oracle as a baseline and the SM clocks seen under load.
+``--impl reference`` times the CPU oracle instead (the only reference
+implementation this operation has here).
 """
 
 from __future__ import annotations
@@ -44,26 +49,27 @@ from mla_decode_attention_10_b200 import workloads as W  # noqa: E402
 
 METRIC = "µs/call and achieved HBM GB/s (fraction of ~8 TB/s) vs T for MLA epilogue"
 UNIT = "µs/call"
-HEADLINE = "split_boundary_t64_h16_rope"
+HEADLINE = "batch_t8192_h16_pdl_fp8"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+REPLAYS = 11          # timed regions per headline measurement (median reported)
+CONTEXT_REPLAYS = 5   # timed regions per context measurement
+DECODE_T = (1, 2, 4, 8, 16, 32, 64)
+IMPLEMENTATION = "CUDA sm_100a kernels through the C ABI (libmla_epilogue.so)"
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the epilogue kernel, from ncu captures of `bench.py --steps 3 --warmup 3
-# --no-sweep --no-cpu-baseline --workload <name>` (third launch; summaries in
-# profiles/).  Keyed by a hash of the kernel sources they were taken on: a
-# changed kernel reports null until it is captured again.
+# --no-sweep --no-cpu-baseline --workload <name>` (summaries in profiles/).
+# Keyed by a hash of the kernel sources they were taken on: a changed kernel
+# reports null until it is captured again.
 KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
+                  "mla_decode_attention_10_b200/csrc/mla_rows.cu",
+                  "mla_decode_attention_10_b200/csrc/epilogue_device.cuh",
                   "mla_decode_attention_10_b200/csrc/latent_math.cuh", "include/mla_epilogue.h")
-TRAFFIC_SOURCE_HASH = "097d8a46e6e610e8"
-TRAFFIC_BYTES = {
-    "split_boundary_t64_h16_rope": 1277952 + 0,
-    "prefill_t1024_h128_strided": 152627456 + 102022400,
-    "batch_t8192_h16_pdl_fp8": 164003328 + 55213568,
-}
+TRAFFIC_SOURCE_HASH = None
+TRAFFIC_BYTES = {}
 L2_BYTES = 126 * 2 ** 20
 GRAPH_CALLS = 500
-
-
 # ---------------------------------------------------------------------------------------
 # ranks
 # ---------------------------------------------------------------------------------------
@@ -335,6 +341,230 @@ def flush_l2():
 # our implementation
 # ---------------------------------------------------------------------------------------
 
+def median_us(runner, device, calls: int, reps: int, world: int = 1, flush: bool = True) -> float:
+    """Median over `reps` timed regions of one replay each, as whole-job
+    microseconds per call (each region's time is the max over ranks)."""
+    return statistics.median(job_us_per_call(timed(runner, device, flush), calls, world) for _ in range(reps))
+
+
+class Harness:
+    """Step functions on one stream: the epilogue on a workload's device sets,
+    the synthetic producer, the empty kernel with the epilogue's grid."""
+
+    def __init__(self, E, stream):
+        self.E = E
+        self.stream = stream
+
+    def epilogue(self, ds, extra=0):
+        E, stream = self.E, self.stream
+
+        def f(i):
+            d, q_out, _ = ds.sets[i % len(ds.sets)]
+            rc = E.launch_workload(d, q_out, extra_flags=extra, stream=stream)
+            if rc != E.MLA_OK:
+                raise E.MlaError(rc, "mla_epilogue_launch")
+        return f
+
+    def empty(self, w0, flags):
+        E, stream = self.E, self.stream
+        plan = E.mla_epilogue_plan(w0.T, w0.H, w0.flags)
+
+        def f(i):
+            rc = E.mla_harness_empty(plan.blocks, plan.threads_per_block, flags, stream.cuda_stream)
+            if rc != E.MLA_OK:
+                raise E.MlaError(rc, "mla_harness_empty")
+        return f, plan
+
+    def producer(self, ds):
+        """The producer writes set i's q_nope / q_pe (from its staged copy, or
+        from the next set's values when the sets carry none: the values do not
+        matter for timing)."""
+        E, stream, S = self.E, self.stream, len(ds.sets)
+
+        def f(i):
+            d, _, src = ds.sets[i % S]
+            if src is None:
+                nxt = ds.sets[(i + 1) % S][0]
+                src = (nxt.q_nope, nxt.q_pe)
+            rc = E.mla_harness_produce(src[0].data_ptr(), src[1].data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0),
+                                       d.q_nope.stride(1), d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1),
+                                       d.T, d.H, 0, stream.cuda_stream)
+            if rc != E.MLA_OK:
+                raise E.MlaError(rc, "mla_harness_produce")
+        return f
+
+    def runner(self, step, calls, warmup=3):
+        warm = GraphRunner(step, max(warmup, 1), self.stream)
+        warm.replay()
+        torch.cuda.synchronize()
+        del warm
+        r = GraphRunner(step, calls, self.stream)
+        r.replay()  # the first replay uploads the graphs
+        torch.cuda.synchronize()
+        return r
+
+
+def then(*fns):
+    def f(i):
+        for g in fns:
+            g(i)
+    return f
+
+
+def behind_producer(hx, ds, device, calls, reps):
+    """Per call: the synthetic producer writes the query inputs, then X is
+    launched as its programmatic dependent (PDL).  X is the epilogue, the
+    empty kernel (same grid) and the empty kernel that executes
+    griddepcontrol.wait; each increment is X's cost over the producer alone.
+    The floor of a dependent launch is the empty kernel that waits: one that
+    does not wait runs beside the producer and is not a dependent at all."""
+    E = hx.E
+    prod = hx.producer(ds)
+    empty, _ = hx.empty(ds.w0, E.MLA_FLAG_PDL)
+    empty_wait, _ = hx.empty(ds.w0, E.MLA_FLAG_PDL | E.MLA_HARNESS_EMPTY_WAIT)
+    steps = {"producer_us": prod,
+             "producer_epilogue_pdl_us": then(prod, hx.epilogue(ds, E.MLA_FLAG_PDL)),
+             "producer_epilogue_no_pdl_us": then(prod, hx.epilogue(ds)),
+             "producer_empty_pdl_us": then(prod, empty),
+             "producer_empty_wait_pdl_us": then(prod, empty_wait)}
+    out = {}
+    for key, fn in steps.items():
+        r = hx.runner(fn, calls)
+        out[key] = round(median_us(r, device, calls, reps), 4)
+        del r
+    p = out["producer_us"]
+    inc = out["producer_epilogue_pdl_us"] - p
+    inc_wait = out["producer_empty_wait_pdl_us"] - p
+    inc_empty = out["producer_empty_pdl_us"] - p
+    out["epilogue_increment_pdl_us"] = round(inc, 4)
+    out["epilogue_increment_no_pdl_us"] = round(out["producer_epilogue_no_pdl_us"] - p, 4)
+    out["empty_wait_increment_us"] = round(inc_wait, 4)
+    out["empty_increment_us"] = round(inc_empty, 4)
+    out["floor_ratio_behind_producer"] = round(inc / inc_wait, 3) if inc_wait > 0 else None
+    return out
+
+
+def standalone(hx, ds, device, calls, reps, peak):
+    """The epilogue alone on cold inputs against the empty kernel of the same
+    grid; `calls` None: 20 calls per region for sizes above 32 MiB, else 200."""
+    w0 = ds.w0
+    if calls is None:
+        calls = 20 if ds.bytes_per_call > 32 * 2 ** 20 else 200
+    r = hx.runner(hx.epilogue(ds), calls)
+    us = median_us(r, device, calls, reps)
+    del r
+    fstep, plan = hx.empty(w0, 0)
+    fr = hx.runner(fstep, calls)
+    floor_us = median_us(fr, device, calls, reps)
+    del fr
+    gbs = w0.algorithmic_bytes() / (us * 1e-6) / 1e9
+    return {"workload": ds.name, "T": w0.T, "H": w0.H, "flags": flag_names(w0.flags), "mode": mode_name(hx.E, plan),
+            "grid": [plan.blocks, plan.threads_per_block], "bytes_per_call": w0.algorithmic_bytes(),
+            "traffic": traffic_for(ds.name), "us_per_call": round(us, 4), "gbs": round(gbs, 1),
+            "frac": round(gbs / peak, 4), "frac_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+            "launch_floor_us": round(floor_us, 4), "floor_ratio": round(us / floor_us, 3), "calls": calls,
+            "sets": len(ds.sets), "l2": f"{ds.touched / 2 ** 20:.0f} MiB touched per rotation"}
+
+
+def mode_name(E, plan):
+    return {E.MLA_MODE_SPLIT: "split", E.MLA_MODE_ROWS: "rows", E.MLA_MODE_TOKEN: "token"}[plan.mode]
+
+
+def decode_floors(hx, device, peak, calls=200, reps=7):
+    """T = 1 .. 64 (the decode sweep workload: H=16, RoPE, e4m3): standalone
+    with cold inputs, and behind the producer with PDL against the floor of
+    a dependent launch."""
+    out = []
+    for T in DECODE_T:
+        ds = DeviceSets(f"decode_sweep_t{T}_h16_rope_fp8")
+        row = standalone(hx, ds, device, calls, reps, peak)
+        row.update(behind_producer(hx, ds, device, calls, reps))
+        out.append(row)
+        del ds
+        torch.cuda.empty_cache()
+    return out
+
+
+def launch_to_end(hx, device, names=("decode_sweep_t1_h16_rope_fp8", "decode_sweep_t4_h16_rope_fp8",
+                                     "decode_sweep_t64_h16_rope_fp8"), iters=1000):
+    """Device time from an event recorded just before one isolated launch to
+    one recorded just after it, for the epilogue and for the empty kernel of
+    the same grid: median (and 10th / 90th percentile) of `iters` launches,
+    each preceded, outside its event pair, by a write of twice the L2 (which
+    also keeps the launch queued ahead of the GPU, so the pair holds the
+    device-side launch, the kernel and its completion, not host overhead)."""
+    E, stream = hx.E, hx.stream
+    buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=device)
+    out = []
+    for name in names:
+        ds = DeviceSets(name)
+        epi = hx.epilogue(ds)
+        empty, plan = hx.empty(ds.w0, 0)
+        row = {"workload": name, "T": ds.w0.T, "H": ds.w0.H, "mode": mode_name(E, plan), "launches": iters}
+        for key, fn in (("epilogue", epi), ("empty", empty)):
+            times = []
+            for base in range(0, iters, 100):
+                pairs = []
+                with torch.cuda.stream(stream):
+                    for i in range(base, min(iters, base + 100)):
+                        buf.fill_(i)
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record(stream)
+                        fn(i)
+                        e1.record(stream)
+                        pairs.append((e0, e1))
+                torch.cuda.synchronize()
+                times += [a.elapsed_time(b) * 1e3 for a, b in pairs]
+            times.sort()
+            row[key] = {"median_us": round(statistics.median(times), 3),
+                        "p10_us": round(times[len(times) // 10], 3), "p90_us": round(times[9 * len(times) // 10], 3)}
+        row["ratio"] = round(row["epilogue"]["median_us"] / row["empty"]["median_us"], 3)
+        out.append(row)
+        del ds
+    del buf
+    torch.cuda.empty_cache()
+    return out
+
+
+def producer_consumer_chain(hx, ds, device, calls, reps):
+    """Per step: the synthetic producer writes a set's q_nope / q_pe, the
+    epilogue runs on that set, and the synthetic consumer reads its q_out and
+    cache rows; timed with the epilogue and the consumer launched as
+    programmatic dependents (PDL) and without."""
+    E, stream = hx.E, hx.stream
+    w0 = ds.w0
+    scores = torch.empty(w0.T * w0.H, dtype=torch.float32, device=device)
+    cflags = (E.MLA_FLAG_Q_FP8 if w0.q_fp8 else 0) | (E.MLA_FLAG_KV_FP8 if w0.kv_fp8 else 0)
+    prod = hx.producer(ds)
+
+    def consume(pdl):
+        def f(i):
+            d, q_out, _ = ds.sets[i % len(ds.sets)]
+            rc = E.mla_harness_consume(q_out.data_ptr(), d.cache.data_ptr(), d.slot_mapping.data_ptr(), d.T, d.H,
+                                       d.num_blocks * d.block_size, cflags | pdl, scores.data_ptr(),
+                                       stream.cuda_stream)
+            if rc != E.MLA_OK:
+                raise E.MlaError(rc, "mla_harness_consume")
+        return f
+
+    out = {"workload": ds.name}
+    for key, fn in (("producer_us", prod),
+                    ("chain_pdl_us", then(prod, hx.epilogue(ds, E.MLA_FLAG_PDL), consume(E.MLA_FLAG_PDL))),
+                    ("chain_no_pdl_us", then(prod, hx.epilogue(ds), consume(0)))):
+        r = hx.runner(fn, calls)
+        out[key] = round(median_us(r, device, calls, reps), 3)
+        del r
+    out["pdl_saves_us"] = round(out["chain_no_pdl_us"] - out["chain_pdl_us"], 3)
+    out["steps"] = calls
+    return out
+
+
+def common_config(name: str):
+    """The `config` both arms print (plus their own `implementation`)."""
+    w = W.RECIPES[name]
+    return {"workload": name, "T": w["T"], "H": w["H"], "flags": flag_names(w["flags"]), "recipe": w["recipe"]}
+
+
 def run_ours(args, rank, world, local_rank):
     from mla_decode_attention_10_b200 import epilogue as E
 
@@ -342,41 +572,15 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     E.lib()  # fail loudly if the CUDA library is missing
     stream = torch.cuda.Stream(device)
+    hx = Harness(E, stream)
     peak, peak_note = measured_hbm_gbs()
 
-    def epilogue_step(ds, extra=0, single_set=False):
-        def f(i):
-            d, q_out, _ = ds.sets[0 if single_set else i % len(ds.sets)]
-            rc = E.launch_workload(d, q_out, extra_flags=extra, stream=stream)
-            if rc != E.MLA_OK:
-                raise E.MlaError(rc, "mla_epilogue_launch")
-        return f
-
-    def floor_step(T, H, flags):
-        plan = E.mla_epilogue_plan(T, H, flags)
-
-        def f(i):
-            rc = E.mla_harness_empty(plan.blocks, plan.threads_per_block, flags & E.MLA_FLAG_PDL, stream.cuda_stream)
-            if rc != E.MLA_OK:
-                raise E.MlaError(rc, "mla_harness_empty")
-        return f, plan
-
-    def measure(step, steps, warmup):
-        warm = GraphRunner(step, max(warmup, 1), stream)
-        warm.replay()
-        torch.cuda.synchronize()
-        runner = GraphRunner(step, steps, stream)
-        runner.replay()  # first replay uploads the graphs
-        torch.cuda.synchronize()
-        return runner
-
-    # ---- headline workload
+    # ---- headline workload: K calls per timed region, REPLAYS regions, median
     ds = DeviceSets(args.workload)
     w0 = ds.w0
-    step = epilogue_step(ds)
-    runner = measure(step, args.steps, args.warmup)
-    fstep, plan = floor_step(w0.T, w0.H, 0)
-    frunner = measure(fstep, args.steps, args.warmup)
+    runner = hx.runner(hx.epilogue(ds), args.steps, args.warmup)
+    fstep, plan = hx.empty(w0, 0)
+    frunner = hx.runner(fstep, args.steps, args.warmup)
     for _ in range(args.warmup):
         runner.replay()
     torch.cuda.synchronize()
@@ -388,92 +592,78 @@ def run_ours(args, rank, world, local_rank):
             runner.replay()
             torch.cuda.synchronize()
         t0 = time.time()
-        ms = timed(runner, device)
+        region_ms = [timed(runner, device) for _ in range(REPLAYS)]
         t1 = time.time()
         time.sleep(0.25)
     clocks = clk.summary(t0, t1)
-    floor_ms = timed(frunner, device)
+    ms = statistics.median(region_ms)
+    floor_us = median_us(frunner, device, args.steps, REPLAYS)
+    del frunner
 
+    l2_note = (f"inputs larger than L2: {len(ds.sets)} rotating input sets touching {ds.touched / 2 ** 20:.0f} MiB "
+               "(> 2x L2); L2 written over before every timed region")
     us = job_us_per_call(ms, args.steps, world)
     per_call_us_rank = ms * 1e3 / args.steps
     gbs = w0.algorithmic_bytes() / (per_call_us_rank * 1e-6) / 1e9
-    floor_us = floor_ms * 1e3 / args.steps
+    spread = [round(x * 1e3 / args.steps, 4) for x in sorted(region_ms)]
 
-    # PDL-chained variant of the same call sequence (each call a programmatic
-    # dependent of the previous one; sets are disjoint, so the contract holds)
-    prunner = measure(epilogue_step(ds, E.MLA_FLAG_PDL), args.steps, args.warmup)
-    pfstep, _ = floor_step(w0.T, w0.H, E.MLA_FLAG_PDL)
-    pfrunner = measure(pfstep, args.steps, args.warmup)
-    pdl_us = timed(prunner, device) * 1e3 / args.steps
-    pdl_floor_us = timed(pfrunner, device) * 1e3 / args.steps
-    del prunner, pfrunner
-
-    # same inputs every call: they stay in L2, as when the upstream kernel has just written them
-    wrunner = measure(epilogue_step(ds, 0, single_set=True), args.steps, args.warmup)
-    warm_us = timed(wrunner, device, flush=False) * 1e3 / args.steps
-    del wrunner
-
-    # producer -> epilogue -> consumer, with and without programmatic dependent launch
-    chain = producer_consumer_chain(ds, E, stream, device, min(args.steps, 500), args.warmup)
+    # the same calls launched as programmatic dependents of the synthetic producer
+    headline_pdl = behind_producer(hx, ds, device, min(args.steps, GRAPH_CALLS), CONTEXT_REPLAYS) if w0.producer \
+        else None
+    del runner
 
     # ---- end to end through the Python API: pinned host inputs -> call -> q_out to host
     e2e = run_e2e(args, w0, stream, device, world)
+    del ds
+    torch.cuda.empty_cache()
 
-    # ---- sweep of the other sizes (their own bench lines are not printed; this is context)
-    # the headline is measured; what follows is context, and an error in it is
-    # reported in the line rather than losing the line
-    sweep = []
-    context_errors = []
-    if not args.no_sweep:
-        for name in sweep_names(args.workload):
-            try:
-                sweep.append(sweep_one(name, E, stream, device, peak, epilogue_step, floor_step, measure))
-            except Exception as exc:  # noqa: BLE001
-                context_errors.append(f"{name}: {type(exc).__name__}: {str(exc).splitlines()[0][:200]}")
-            torch.cuda.empty_cache()
+    # ---- context: decode sizes, launch-to-end latency, other sizes, PDL chain, absorbed query rows
+    context, context_errors = {}, []
 
-    absorb = None
-    if not args.no_sweep:
+    def ctx(key, fn):
         try:
-            absorb = absorb_measure(E, stream, device, peak)
-        except Exception as exc:  # noqa: BLE001
-            context_errors.append(f"absorbed_query: {type(exc).__name__}: {str(exc).splitlines()[0][:200]}")
+            context[key] = fn()
+        except Exception as exc:  # noqa: BLE001 -- context only: report, keep the line
+            context_errors.append(f"{key}: {type(exc).__name__}: {str(exc).splitlines()[0][:200]}")
+        torch.cuda.empty_cache()
 
+    if not args.no_sweep:
+        ctx("decode_floors", lambda: decode_floors(hx, device, peak))
+        ctx("launch_to_end", lambda: launch_to_end(hx, device))
+        ctx("sweep", lambda: [standalone(hx, DeviceSets(n), device, None, CONTEXT_REPLAYS, peak)
+                              for n in sweep_names(args.workload)])
+        ctx("producer_epilogue_consumer",
+            lambda: producer_consumer_chain(hx, DeviceSets("split_boundary_t64_h16_rope"), device, 200,
+                                            CONTEXT_REPLAYS))
+        ctx("absorbed_query", lambda: absorb_measure(E, stream, device, peak))
+
+    config = dict(common_config(args.workload), implementation=IMPLEMENTATION)
     line = {
         "metric": METRIC, "value": round(us, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "T": w0.T, "H": w0.H, "flags": flag_names(w0.flags),
-                   "recipe": w0.recipe, "mode": "split" if plan.mode == E.MLA_MODE_SPLIT else "rows",
-                   "grid": [plan.blocks, plan.threads_per_block],
-                   "l2": f"inputs larger than L2: {len(ds.sets)} rotating input sets touching "
-                         f"{ds.touched / 2 ** 20:.0f} MiB (> 2x L2); L2 written over before each timed region",
-                   "timing": f"CUDA graphs of <= {GRAPH_CALLS} calls on one stream, CUDA events",
+        "config": config,
+        "timing": {"mode": mode_name(E, plan), "grid": [plan.blocks, plan.threads_per_block],
+                   "regions": REPLAYS, "region_us_per_call_sorted": spread,
+                   "l2": l2_note,
+                   "method": f"median of {REPLAYS} timed regions, each one replay of CUDA graphs holding the "
+                             f"{args.steps} calls (<= {GRAPH_CALLS} per graph) on one stream, CUDA events on that "
+                             "stream, barrier + synchronize around each region",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "gbs": round(gbs, 1),
         "launch_floor_us": round(floor_us, 4),
         "floor_ratio": round(per_call_us_rank / floor_us, 3),
-        "pdl_chain": {"us_per_call": round(pdl_us, 4), "floor_us": round(pdl_floor_us, 4),
-                      "floor_ratio": round(pdl_us / pdl_floor_us, 3),
-                      "note": "each call a programmatic dependent of the previous one (disjoint input sets)"},
-        "l2_warm": {"us_per_call": round(warm_us, 4), "floor_ratio": round(warm_us / floor_us, 3),
-                    "note": "the same inputs every call, so they are L2-resident (not the headline: the "
-                            "headline reads HBM)"},
-        "producer_epilogue_consumer": chain,
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "traffic": traffic_for(args.workload),
-                     "algorithmic_bytes": w0.algorithmic_bytes(),
-                     "peak_source": peak_note,
-                     "note": "decode-size call: launch and memory latency bound, not bandwidth bound; "
-                             "see sweep for the bandwidth-bound sizes. traffic counts DRAM bytes inside the "
-                             "launch: written rows stay in L2 (write-back) and reach DRAM later"},
+                     "algorithmic_bytes": w0.algorithmic_bytes(), "peak_source": peak_note,
+                     "frac_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)},
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clocks,
-        "sweep": sweep,
     }
-    if absorb is not None:
-        line["absorbed_query"] = absorb
+    if headline_pdl is not None:
+        line["behind_producer"] = headline_pdl
+    line.update(context)
     if context_errors:
         line["context_errors"] = context_errors
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -489,117 +679,10 @@ def flag_names(f: int) -> str:
 
 
 def sweep_names(headline: str):
-    names = ["decode_t4_h16", "split_boundary_t64_h16_rope", "split_boundary_t65_h16_rope"]
-    names += [f"decode_sweep_t{t}_h16_rope_fp8" for t in W.DECODE_SWEEP_T]
-    names += ["prefill_t1024_h128_strided", "batch_t8192_h16_pdl_fp8"]
+    names = ["decode_t4_h16", "split_boundary_t64_h16_rope", "split_boundary_t65_h16_rope",
+             "decode_sweep_t128_h16_rope_fp8", "decode_sweep_t256_h16_rope_fp8",
+             "prefill_t1024_h128_strided", "batch_t8192_h16_pdl_fp8"]
     return [n for n in names if n != headline]
-
-
-def sweep_one(name, E, stream, device, peak, epilogue_step, floor_step, measure, steps=None):
-    ds = DeviceSets(name)
-    w0 = ds.w0
-    big = w0.algorithmic_bytes() > 32 * 2 ** 20
-    n = steps or (20 if big else max(1000, len(ds.sets)))
-    r = measure(epilogue_step(ds), n, 3)
-    us = timed(r, device) * 1e3 / n
-    fstep, plan = floor_step(w0.T, w0.H, 0)
-    fr = measure(fstep, n, 3)
-    floor_us = timed(fr, device) * 1e3 / n
-    gbs = w0.algorithmic_bytes() / (us * 1e-6) / 1e9
-    out = {"workload": name, "T": w0.T, "H": w0.H, "flags": flag_names(w0.flags),
-           "mode": "split" if plan.mode == E.MLA_MODE_SPLIT else "rows",
-           "bytes_per_call": w0.algorithmic_bytes(), "traffic": traffic_for(name), "us_per_call": round(us, 3),
-           "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "launch_floor_us": round(floor_us, 3),
-           "floor_ratio": round(us / floor_us, 3), "calls": n, "sets": len(ds.sets),
-           "l2": f"{ds.touched / 2 ** 20:.0f} MiB touched per rotation"}
-    if w0.producer:
-        out.update(producer_pdl(ds, E, stream, device, n))
-    del r, fr
-    return out
-
-
-def producer_pdl(ds, E, stream, device, n):
-    """Producer alone vs producer + epilogue launched with PDL behind it."""
-    def prod(i):
-        d, _, (sn, sp) = ds.sets[i % len(ds.sets)]
-        rc = E.mla_harness_produce(sn.data_ptr(), sp.data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0),
-                                   d.q_nope.stride(1), d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1),
-                                   d.T, d.H, 0, stream.cuda_stream)
-        assert rc == E.MLA_OK
-
-    def pair(i):
-        prod(i)
-        d, q_out, _ = ds.sets[i % len(ds.sets)]
-        rc = E.launch_workload(d, q_out, extra_flags=E.MLA_FLAG_PDL, stream=stream)
-        assert rc == E.MLA_OK
-
-    def pair_nopdl(i):
-        prod(i)
-        d, q_out, _ = ds.sets[i % len(ds.sets)]
-        rc = E.launch_workload(d, q_out, stream=stream)
-        assert rc == E.MLA_OK
-
-    res = {}
-    for key, fn in (("producer_us", prod), ("producer_plus_epilogue_pdl_us", pair),
-                    ("producer_plus_epilogue_no_pdl_us", pair_nopdl)):
-        g = GraphRunner(fn, n, stream)
-        g.replay()
-        torch.cuda.synchronize()
-        res[key] = round(timed(g, device) * 1e3 / n, 3)
-        del g
-    res["epilogue_increment_pdl_us"] = round(res["producer_plus_epilogue_pdl_us"] - res["producer_us"], 3)
-    return res
-
-
-def producer_consumer_chain(ds, E, stream, device, n, warmup):
-    """Per step: the synthetic producer writes a set's q_nope / q_pe, the
-    epilogue runs on that set, and the synthetic consumer reads its q_out and
-    cache rows.  Timed with the epilogue and the consumer launched as
-    programmatic dependents (PDL) and without; `producer_us` alone for
-    reference.  Values do not matter here (the producer copies the next
-    set's query inputs); stream order keeps every step after the last."""
-    S = len(ds.sets)
-    w0 = ds.w0
-    scores = torch.empty(w0.T * w0.H, dtype=torch.float32, device=device)
-    cflags = (E.MLA_FLAG_Q_FP8 if w0.q_fp8 else 0) | (E.MLA_FLAG_KV_FP8 if w0.kv_fp8 else 0)
-
-    sources = {}
-
-    def source(k):
-        # the producer reads contiguous [T,H,512] / [T,H,64] buffers
-        if k not in sources:
-            d, _, src = ds.sets[k]
-            sources[k] = src if src is not None else (d.q_nope.contiguous(), d.q_pe.contiguous())
-        return sources[k]
-
-    def prod(i):
-        d, _, _ = ds.sets[i % S]
-        sn, sp = source((i + 1) % S) if ds.sets[i % S][2] is None else source(i % S)
-        rc = E.mla_harness_produce(sn.data_ptr(), sp.data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0),
-                                   d.q_nope.stride(1), d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1),
-                                   d.T, d.H, 0, stream.cuda_stream)
-        assert rc == E.MLA_OK
-
-    def chain(pdl):
-        def f(i):
-            prod(i)
-            d, q_out, _ = ds.sets[i % S]
-            assert E.launch_workload(d, q_out, extra_flags=pdl, stream=stream) == E.MLA_OK
-            assert E.mla_harness_consume(q_out.data_ptr(), d.cache.data_ptr(), d.slot_mapping.data_ptr(), d.T, d.H,
-                                         d.num_blocks * d.block_size, cflags | pdl, scores.data_ptr(),
-                                         stream.cuda_stream) == E.MLA_OK
-        return f
-
-    out = {}
-    for key, fn in (("producer_us", prod), ("chain_pdl_us", chain(E.MLA_FLAG_PDL)), ("chain_no_pdl_us", chain(0))):
-        g = GraphRunner(fn, n, stream)
-        g.replay()
-        torch.cuda.synchronize()
-        out[key] = round(timed(g, device) * 1e3 / n, 3)
-        del g
-    out["pdl_saves_us"] = round(out["chain_no_pdl_us"] - out["chain_pdl_us"], 3)
-    out["steps"] = n
-    return out
 
 
 def absorb_measure(E, stream, device, peak_gbs):
@@ -607,7 +690,6 @@ def absorb_measure(E, stream, device, peak_gbs):
     at T=8192, H=16, RoPE, e4m3, against the same work unfused: a cuBLAS
     batched matmul writing the 512-wide product, then the epilogue (which
     also writes the cache rows)."""
-    peak_tf = None
     try:
         peak_tf = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
     except (OSError, KeyError, ValueError):
@@ -622,13 +704,15 @@ def absorb_measure(E, stream, device, peak_gbs):
 
     def fused(i):
         w, q = sets[i % 2]
-        assert E.launch_absorb_workload(w, q, stream=stream) == E.MLA_OK
+        rc = E.launch_absorb_workload(w, q, stream=stream)
+        if rc != E.MLA_OK:
+            raise E.MlaError(rc, "mla_absorb_launch")
 
     n = 20
     r = GraphRunner(fused, n, stream)
     r.replay()
     torch.cuda.synchronize()
-    us = min(timed(r, device) for _ in range(3)) * 1e3 / n
+    us = median_us(r, device, n, CONTEXT_REPLAYS)
     del r
     # unfused: torch.bmm (cuBLAS) for the product, then the epilogue on it
     e_sets = []
@@ -648,7 +732,9 @@ def absorb_measure(E, stream, device, peak_gbs):
     def unfused(i):
         bmm_only(i)
         _, ew, _, q = e_sets[i % 2]
-        assert E.launch_workload(ew, q, stream=stream) == E.MLA_OK
+        rc = E.launch_workload(ew, q, stream=stream)
+        if rc != E.MLA_OK:
+            raise E.MlaError(rc, "mla_epilogue_launch")
 
     # cuBLAS creates its handle and workspace on first use, which cannot happen inside a graph capture
     bmm_only(0)
@@ -658,7 +744,7 @@ def absorb_measure(E, stream, device, peak_gbs):
         g = GraphRunner(fn, n, stream)
         g.replay()
         torch.cuda.synchronize()
-        out[key] = round(min(timed(g, device) for _ in range(3)) * 1e3 / n, 3)
+        out[key] = round(median_us(g, device, n, CONTEXT_REPLAYS), 3)
         del g
     gbs = w0.algorithmic_bytes() / (us * 1e-6) / 1e9
     tfs = w0.flops() / (us * 1e-6) / 1e12
@@ -679,15 +765,12 @@ def run_e2e(args, w0, stream, device, world):
     16-byte aligned offsets, so each step is one host-to-device copy, the
     call, and one device-to-host copy.
 
-    Three schedules are timed.  Serial: all three on the launch stream, one
-    step after the other.  Pipelined (the reported value: the user-facing
-    call is made every step): uploads, calls and downloads on three streams
-    with two buffer sets, the way a serving loop overlaps them: step i+1's
-    upload runs while step i computes and step i-1's result comes back;
-    events order every reuse of a buffer.  Graphed (context): the pipelined
-    schedule of 20 steps captured once as a CUDA graph, with its copy nodes,
-    and replayed, as decode loops launch their steps; every replayed step
-    still moves its inputs and its result over the host link."""
+    Two schedules.  Serial: all three on the launch stream, one step after
+    the other.  Pipelined (the reported value; the user-facing call is made
+    every step): uploads, calls and downloads on three streams over two
+    buffer sets, the way a serving loop overlaps them: step i+1's upload runs
+    while step i computes and step i-1's result comes back; events order
+    every reuse of a buffer."""
     from mla_decode_attention_10_b200 import epilogue as E
     parts = [(k, getattr(w0, k).contiguous()) for k in ("q_nope", "q_pe", "kv_c", "k_pe", "slot_mapping", "positions")
              if getattr(w0, k) is not None]
@@ -722,7 +805,7 @@ def run_e2e(args, w0, stream, device, world):
             dev["q_nope"], dev["q_pe"], dev["kv_c"], dev["k_pe"], cache, dev["slot_mapping"],
             positions=dev.get("positions"), cos_sin=cos_sin, q_scale=qs, kv_scale=ks, q_out=b["q_out"], stream=s)
 
-    def serial_step():
+    def serial_step(i):
         b = sets[0]
         with torch.cuda.stream(stream):
             b["dbuf"].copy_(b["host"], non_blocking=True)
@@ -735,16 +818,14 @@ def run_e2e(args, w0, stream, device, world):
         for n in e:
             e[n].record(stream)
 
-    def pipelined_step(i, first=False):
+    def pipelined_step(i):
         b, e = sets[i % 2], ev[i % 2]
-        if not first:
-            up.wait_event(e["comp"])   # the call two steps back has read this input buffer
+        up.wait_event(e["comp"])   # the call two steps back has read this input buffer
         with torch.cuda.stream(up):
             b["dbuf"].copy_(b["host"], non_blocking=True)
         e["up"].record(up)
         stream.wait_event(e["up"])
-        if not first:
-            stream.wait_event(e["down"])  # the download two steps back has read this q_out
+        stream.wait_event(e["down"])  # the download two steps back has read this q_out
         call(b, stream)
         e["comp"].record(stream)
         down.wait_event(e["comp"])
@@ -768,128 +849,113 @@ def run_e2e(args, w0, stream, device, world):
         barrier(device)
         return max_over_ranks(e0.elapsed_time(e1), device)
 
-    k = max(10, min(args.steps, 200))
-    for _ in range(max(args.warmup, 3)):
-        serial_step()
-    serial_ms = timed_run(lambda i: serial_step(), k)
+    k = max(10, min(args.steps, 100))
+    for i in range(max(args.warmup, 3)):
+        serial_step(i)
+    serial_ms = timed_run(serial_step, k)
     for i in range(max(args.warmup, 3)):
         pipelined_step(i)
     pipe_ms = timed_run(pipelined_step, k)
-    # the same schedule as one CUDA graph of G steps (the first two steps of
-    # a replay wait for nothing: the previous replay has completed)
-    G = 20
-    graph_ms, graph_note, g = None, None, None
-    try:
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            up.wait_stream(stream)
-            down.wait_stream(stream)
-            for i in range(G):
-                pipelined_step(i, first=i < 2)
-            stream.wait_stream(up)
-            stream.wait_stream(down)
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                g.replay()
-        torch.cuda.synchronize()
-    except RuntimeError as exc:  # capture refused: report the stream-pipelined figure
-        graph_note = f"graph capture failed: {exc}"[:200]
-        g = None
-    # every rank takes the same branch, so the collectives inside timed_run match
-    if max_over_ranks(0.0 if g is not None else 1.0, device) == 0.0:
-        reps = max(1, k // G)
-
-        def replay(i):
-            with torch.cuda.stream(stream):
-                g.replay()
-
-        graph_ms = timed_run(replay, reps)
-        graph_steps = G * reps
-    elif graph_note is None:
-        graph_note = "graph capture failed on another rank"
-    out = {"value": round(job_us_per_call(pipe_ms, k, world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": round(job_us_per_call(pipe_ms, k, world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": k,
-            "graphed_value": (round(job_us_per_call(graph_ms, graph_steps, world), 3)
-                              if graph_ms is not None else None),
             "serial_value": round(job_us_per_call(serial_ms, k, world), 3),
             "path": "epilogue.fused_mla_decode_q_concat_kv_cache_insert; per step one host-to-device copy of the "
                     "inputs from a pinned staging buffer, the call, and q_out back to pinned host memory; value: "
                     "uploads, calls and downloads pipelined on three streams over two buffer sets, the call made "
-                    "every step; graphed_value: the same schedule captured as a CUDA graph of 20 steps and "
-                    "replayed; serial_value: all on the launch stream, one step after the other"}
-    if graph_note:
-        out["note"] = graph_note
-    return out
+                    "every step; serial_value: all on the launch stream, one step after the other"}
 
 
 # ---------------------------------------------------------------------------------------
 # CPU oracle: the baseline and the reference arm
 # ---------------------------------------------------------------------------------------
 
-def _oracle_call(w):
+def _oracle_call(w, threads=1):
     import oracle
     return oracle.run(w.q_nope, w.q_pe, w.kv_c, w.k_pe, w.slot_mapping, w.cache, w.flags,
-                      positions=w.positions, cos_sin=w.cos_sin, q_scale=w.q_scale, kv_scale=w.kv_scale)
+                      positions=w.positions, cos_sin=w.cos_sin, q_scale=w.q_scale, kv_scale=w.kv_scale,
+                      threads=threads)
 
 
-def cpu_baseline(name: str, seconds: float = 10.0):
-    """The single-threaded CPU oracle, as it stands, repeated on the workload
-    for about `seconds` of host time."""
-    w = named_variant(name, 0)
-    _oracle_call(w)
+def token_slice(w: W.Workload, n: int) -> W.Workload:
+    """The first n tokens of a workload (same cache, table and scales): a
+    bounded sample of the same work, n/T of a call."""
+    if n >= w.T:
+        return w
+    import dataclasses
+    return dataclasses.replace(w, T=n, q_nope=w.q_nope[:n], q_pe=w.q_pe[:n], kv_c=w.kv_c[:n], k_pe=w.k_pe[:n],
+                               slot_mapping=w.slot_mapping[:n],
+                               positions=None if w.positions is None else w.positions[:n])
+
+
+def sampled_oracle(w: W.Workload, seconds: float, threads: int = 1):
+    """Time the oracle, as it stands, on token slices of `w` for about
+    `seconds` of host time; returns (µs per full call, calls, tokens per call)."""
+    probe = token_slice(w, max(1, w.T // 16))
+    t0 = time.perf_counter()
+    _oracle_call(probe, threads)
+    est_full = (time.perf_counter() - t0) * w.T / probe.T
+    n_tok = w.T if est_full <= seconds / 4 else max(1, int(w.T * seconds / 4 / est_full))
+    s = token_slice(w, n_tok)
     n, t0 = 0, time.perf_counter()
-    while time.perf_counter() - t0 < seconds:
-        _oracle_call(w)
+    while time.perf_counter() - t0 < seconds or n == 0:
+        _oracle_call(s, threads)
         n += 1
     dt = time.perf_counter() - t0
-    return {"value": round(dt / n * 1e6, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} calls of {name} (T={w.T}, H={w.H}) in {dt:.1f} s, one host thread "
-                      f"({os.cpu_count()} cores on the host)"}
+    return dt / n * 1e6 * w.T / n_tok, n, n_tok
 
 
-def cpu_baseline_all_cores(name: str, seconds: float = 5.0):
+def cpu_baseline(name: str, seconds: float = 12.0):
+    """The single-threaded CPU oracle, as it stands, on token slices of the
+    workload for about `seconds` of host time, scaled to one full call."""
+    w = named_variant(name, 0)
+    us, n, n_tok = sampled_oracle(w, seconds)
+    return {"value": round(us, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} calls on {n_tok} of the {w.T} tokens of {name} (H={w.H}) in ~{seconds:.0f} s, one host "
+                      f"thread, scaled by {w.T}/{n_tok} ({os.cpu_count()} cores on the host)"}
+
+
+def cpu_baseline_all_cores(name: str, seconds: float = 6.0):
     """The same oracle function, as it stands, on contiguous token slices on
     every host core at once (one std::thread per slice inside the oracle
     library).  Reported as a baseline only."""
-    import oracle
     w = named_variant(name, 0)
     cores = max(1, min(os.cpu_count() or 1, w.T))
-
-    def call():
-        oracle.run(w.q_nope, w.q_pe, w.kv_c, w.k_pe, w.slot_mapping, w.cache, w.flags, positions=w.positions,
-                   cos_sin=w.cos_sin, q_scale=w.q_scale, kv_scale=w.kv_scale, threads=cores)
-
-    call()
-    n, t0 = 0, time.perf_counter()
-    while time.perf_counter() - t0 < seconds:
-        call()
-        n += 1
-    dt = time.perf_counter() - t0
-    return {"value": round(dt / n * 1e6, 2), "unit": UNIT, "cores": cores, "kind": "oracle, token slices on threads",
-            "sample": f"{n} calls of {name} (T={w.T}, H={w.H}) in {dt:.1f} s, {cores} threads of "
-                      f"{-(-w.T // cores)} tokens at most; baseline only"}
+    us, n, n_tok = sampled_oracle(w, seconds, threads=cores)
+    return {"value": round(us, 2), "unit": UNIT, "cores": cores, "kind": "oracle, token slices on threads",
+            "sample": f"{n} calls on {n_tok} of the {w.T} tokens of {name} in ~{seconds:.0f} s, {cores} threads, "
+                      f"scaled by {w.T}/{n_tok}; baseline only"}
 
 
-def run_reference(args, rank, world):
+def run_reference(args, rank, world, budget_s: float = 150.0):
+    """The oracle as the reference arm: every step a token slice of the
+    workload sized so that warm-up and timed steps together take about
+    `budget_s` seconds at most, its time scaled to a full call."""
     if rank != 0:
         return None
     w = named_variant(args.workload, 0)
+    probe = token_slice(w, max(1, w.T // 16))
+    t0 = time.perf_counter()
+    _oracle_call(probe)
+    est_full = (time.perf_counter() - t0) * w.T / probe.T
+    per_step = budget_s / (args.steps + args.warmup)
+    n_tok = w.T if est_full <= per_step else max(1, int(w.T * per_step / est_full))
+    s = token_slice(w, n_tok)
     for _ in range(args.warmup):
-        _oracle_call(w)
+        _oracle_call(s)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_call(w)
+        _oracle_call(s)
     dt = time.perf_counter() - t0
-    us = dt / args.steps * 1e6
-    cb = {"value": round(us, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-          "sample": f"{args.steps} calls of {args.workload} (T={w.T}, H={w.H}), one host thread"}
+    us = dt / args.steps * 1e6 * w.T / n_tok
+    sample = (f"{args.steps} steps, each the oracle on {n_tok} of the {w.T} tokens of {args.workload} (H={w.H}), "
+              f"one host thread, scaled by {w.T}/{n_tok}")
+    cb = {"value": round(us, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
     return {"impl": "reference", "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": args.workload, "T": w.T, "H": w.H, "flags": flag_names(w.flags),
-                       "recipe": w.recipe, "implementation": "CPU oracle (oracle/mla_oracle.cpp)"},
+            "config": dict(common_config(args.workload), implementation="CPU oracle (oracle/mla_oracle.cpp), "
+                                                                        "one host thread"),
             "cpu_baseline": cb,
             "e2e": {"value": round(us, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -899,8 +965,8 @@ def run_reference(args, rank, world):
 def parse(argv=None):
     p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
-    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default=HEADLINE, choices=W.names())
     p.add_argument("--no-sweep", action="store_true")

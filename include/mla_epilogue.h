@@ -63,16 +63,20 @@ typedef enum mla_status {
 #define MLA_FLAG_Q_FP8       2u  /* q_out is e4m3 bytes, scaled by *q_scale (needs q_scale) */
 #define MLA_FLAG_KV_FP8      4u  /* cache is e4m3 bytes, scaled by *kv_scale (needs kv_scale) */
 #define MLA_FLAG_PDL         8u  /* launch as a programmatic dependent of the previous kernel on `stream` */
-#define MLA_FLAG_FORCE_SPLIT 16u /* use the small-batch kernel whatever T is (tests, tuning) */
-#define MLA_FLAG_FORCE_ROWS  32u /* use the large-batch kernel whatever T is (tests, tuning) */
+#define MLA_FLAG_FORCE_SPLIT 16u /* use MLA_MODE_SPLIT whatever T is (tests, tuning) */
+#define MLA_FLAG_FORCE_ROWS  32u /* use MLA_MODE_ROWS whatever T is (tests, tuning) */
+#define MLA_FLAG_FORCE_TOKEN 64u /* use MLA_MODE_TOKEN whatever T is (tests, tuning); at most one FORCE flag */
 
 /* bits the kernel ORs into *status */
 #define MLA_STATUS_SLOT_RANGE 1  /* some slot_mapping[t] >= num_blocks*block_size: that cache row was not written */
 #define MLA_STATUS_POS_RANGE  2  /* some positions[t] outside [0, rope_rows): that token's rows were not rotated */
 
 /* Kernel choice (mla_plan.mode). */
-#define MLA_MODE_SPLIT 1 /* three warps per 576-wide row, one 16-byte chunk (or one RoPE pair) per lane */
-#define MLA_MODE_ROWS  2 /* one warp per row, several rows in flight per warp, grid a multiple of the SM count */
+#define MLA_MODE_SPLIT 1 /* small T: 68 threads per 576-wide row, 64 with one 16-byte nope chunk each and 4 with
+                            eight RoPE pairs each (16-byte loads); rows_per_block rows per block */
+#define MLA_MODE_ROWS  2 /* large T: persistent blocks, grid a multiple of the SM count */
+#define MLA_MODE_TOKEN 3 /* T == 1: 36 threads per row (two nope chunks each), every row of the token in one
+                            block when H + 1 <= 28 */
 
 /*
  * mla_epilogue_launch -- the whole epilogue in one kernel launch.
@@ -149,13 +153,13 @@ MLA_API mla_status mla_epilogue_launch(
  * the current device, without launching anything.  Host only; needs the
  * device's SM count, which it reads once per device (sm_count <= 0 lets the
  * caller pass it instead: `sm_count` > 0 is used as given and no CUDA call is
- * made).  Returns MLA_ERR_INVALID_ARG for T < 1, H < 1 or both FORCE flags.
+ * made).  Returns MLA_ERR_INVALID_ARG for T < 1, H < 1 or more than one FORCE flag.
  */
 typedef struct mla_plan {
   int32_t mode;              /* MLA_MODE_SPLIT or MLA_MODE_ROWS */
   int32_t threads_per_block;
   int64_t blocks;
-  int32_t rows_per_block;    /* SPLIT: rows one block covers; ROWS: rows one warp keeps in flight */
+  int32_t rows_per_block;    /* SPLIT, TOKEN: rows one block covers; ROWS: 1 */
   int32_t sm_count;
 } mla_plan;
 
@@ -171,7 +175,7 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  * default threshold counts rows, not tokens.  A value <= 0 keeps the current
  * setting.
  *   split_max_rows       T * (H + 1) at or below which MLA_MODE_SPLIT is used (default 4608)
- *   split_rows_per_block rows per block in MLA_MODE_SPLIT (block = 96 * this), at most 4
+ *   split_rows_per_block rows per block in MLA_MODE_SPLIT (block = 68 * this), at most 15
  *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
  *                        the number the kernel's register cap keeps resident

@@ -40,8 +40,12 @@ MLA_API mla_status mla_harness_produce(const void* src_nope, const void* src_pe,
 /*
  * An empty kernel launched with `blocks` x `threads` and, with MLA_FLAG_PDL,
  * the programmatic-serialization attribute: the bare-launch floor that the
- * epilogue's latency at decode sizes is compared with.
+ * epilogue's latency at decode sizes is compared with.  With
+ * MLA_HARNESS_EMPTY_WAIT every thread executes griddepcontrol.wait and then
+ * exits: the cheapest kernel that honours a programmatic dependency, i.e. the
+ * floor of a dependent launch behind an upstream kernel.
  */
+#define MLA_HARNESS_EMPTY_WAIT 256u
 MLA_API mla_status mla_harness_empty(int64_t blocks, int32_t threads, uint32_t flags, mla_stream_t stream);
 
 /*

@@ -32,11 +32,13 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cstdint>
 
 #include "latent_math.cuh"
 #include "mla_absorb.h"
+#include "mla_runtime.h"
 
 namespace mla {
 namespace absorb {
@@ -591,6 +593,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// Whether the kernel for flag bits k has its shared-memory opt-in on device
+// `dev` (cudaFuncSetAttribute applies per device).
+std::atomic<bool> g_smem_ready[kMaxDevices][4];
+
 }  // namespace absorb
 }  // namespace mla
 
@@ -618,8 +624,12 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
       (status != nullptr && !aligned(status, 4)))
     return MLA_ERR_ALIGNMENT;
 
+  int dev = 0;
+  int32_t sms = 0;
+  const mla_status ds = mla::current_device(&dev, &sms);
+  if (ds != MLA_OK) return ds;
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-  if (encode == nullptr) return MLA_ERR_CUDA;
+  if (encode == nullptr) return mla::cuda_failure(cudaErrorNotSupported);
 
   // A: q_nope_c as (k, h, t), box (64, 1, 128); a size-1 dimension gets any
   // legal stride (it is never stepped over)
@@ -680,23 +690,16 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
   const int k = (qf8 ? 2 : 0) | (rope ? 1 : 0);
   static const void* const kernels[4] = {kernel_for<false, false>(), kernel_for<false, true>(),
                                          kernel_for<true, false>(), kernel_for<true, true>()};
-  static bool smem_set[4] = {false, false, false, false};
   const void* fn = kernels[k];
-  if (!smem_set[k]) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes)) !=
-        cudaSuccess) {
-      (void)cudaGetLastError();
-      return MLA_ERR_CUDA;
-    }
-    smem_set[k] = true;
+  if (!g_smem_ready[dev][k].load(std::memory_order_acquire)) {
+    // idempotent: two threads racing here both set the same attribute
+    const cudaError_t e =
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return mla::cuda_failure(e);
+    g_smem_ready[dev][k].store(true, std::memory_order_release);
   }
 
   cudaLaunchConfig_t cfg = {};
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
   const int64_t tiles = 2 * H * ((T + kM - 1) / kM);
   cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -711,10 +714,7 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
   }
   void* args[] = {&tmA, &tmB, &tmC, &prm};
   const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
+  if (e != cudaSuccess) return mla::cuda_failure(e);
   return MLA_OK;
 }
 

@@ -1,114 +1,51 @@
-// mla_epilogue.cu -- the fused MLA decode epilogue for B200 (sm_100a) and its C-ABI launcher.
+// mla_epilogue.cu -- the fused MLA decode epilogue for B200 (sm_100a): the
+// small-batch kernels and the C-ABI launcher.
 //
 // Per token t: H latent query rows q_out[t, h] = enc(rope(q_nope[t, h] || q_pe[t, h]))
 // and one latent cache row cache[slot_mapping[t]] = enc(rope(kv_c[t] || k_pe[t])),
 // each 576 = 512 + 64 wide (vLLM PR #54896 report, 实现拆解 items 1-3 and the
 // fusedKimiK3MLADecodeQConcatKVCacheKernel / writeLatent576 listing).
 //
-// The op moves bytes and does almost no arithmetic, so it is bound by HBM
-// bandwidth at large T and by launch and memory latency at decode sizes; there
-// is no contraction and no tensor-core work.  Two kernels share the element
-// code (latent_math.cuh):
+// The op moves bytes and does almost no arithmetic: at decode sizes it is
+// bound by launch and memory latency, at large T by HBM bandwidth; there is
+// no contraction and no tensor-core work.  Three launch modes:
 //
-//   split kernel (small T): each row gets three warps, as the page's SPLIT=3
-//     path does.  Warps 0 and 1 copy/convert the 64 nope chunks (16 bytes, 8
-//     values, one chunk per lane); warp 2 does the 64 pe values as 32 RoPE
-//     pairs (i, i+32), one pair per lane, so the rotation needs no shuffles.
-//     Every lane issues its loads at once: the critical path is one
-//     dependent load (position -> table row) plus the data load.
-//   rows kernel (large T): one warp per row (lane: nope chunks lane and
-//     lane+32, pe pair lane); the grid is a multiple of the SM count sized to
-//     the resident blocks, each warp walks a contiguous range of rows, keeps
-//     the next row's loads in flight while it converts the current one, and
-//     looks up a token's rotation once for all of its adjacent rows.
+//   SPLIT (small T): every row gets 68 threads.  64 of them move one 16-byte
+//     nope chunk each (8 values); 4 of them each own the pe octets 8j..8j+7
+//     and 32+8j..32+8j+7, so one thread holds both members of its 8 RoPE
+//     pairs (i, i+32) and rotates them without shuffles, with 16-byte loads
+//     and 16-byte (bf16) or 8-byte (e4m3) stores.  A block holds R rows:
+//     first the 64R nope threads, then the 4R pe threads, so every warp has
+//     one role.
+//   TOKEN (T == 1): the same row code with 32 nope threads per row, two
+//     chunks each (c and c + 32), so all H + 1 rows of the token fit in one
+//     block for H <= 27: one block, one position, one table row, a single
+//     wave of loads (the num_tokens == 1 case of PR #53526, 关联脉络).
+//   ROWS (large T): mla_rows.cu.
 //
-// Row order: rows [0, T) are the T cache rows, rows [T, T + T*H) the query
-// rows in q_out order.  Cache rows never wait on the upstream kernel, so
-// under programmatic dependent launch they run while it finishes
-// (PR #54896 report, 实现拆解 item 2); query rows execute griddepcontrol.wait
-// right before they read q_nope / q_pe, after their slot, position, table and
-// scale loads.  Every thread issues griddepcontrol.launch_dependents after its
-// last store (the report's 评论区精华: the early trigger was a race).
+// In SPLIT and TOKEN every thread computes its addresses and loads its slot,
+// position, table entries and scale before griddepcontrol.wait; after the
+// wait a query-row thread has one load -> convert -> store left (PR #54896
+// report, 实现拆解 item 2).  Cache rows never wait.  Every thread issues
+// griddepcontrol.launch_dependents after its last store (the report's
+// 评论区精华: the early trigger was a race).
 
+#include <atomic>
 #include <climits>
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "latent_math.cuh"
+#include "epilogue_device.cuh"
 #include "mla_epilogue.h"
+#include "mla_rows.h"
+#include "mla_runtime.h"
 
 namespace mla {
 
-constexpr int kNope = 512;
-constexpr int kPe = 64;
-constexpr int kHalfPe = 32;
-constexpr int kRow = 576;
-constexpr int kSplitThreadsPerRow = 96;
-constexpr int kSplitMaxRowsPerBlock = 4;  // 384 threads
-// Resident 256-thread blocks per SM the rows kernel is compiled for: 5 (a
-// 48-register cap) for bf16 outputs; 6 (40 registers) when an output is
-// e4m3, whose arithmetic leaves the kernel short of memory parallelism at 5
-// (measured on B200: 0.75 -> 0.78 of copy bandwidth for T=8192, H=16; the
-// bf16 variants lose at 6).
-constexpr int kRowsMaxBlocksPerSm = 6;
-constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 6 : 5; }
-
-struct Args {
-  const uint16_t* q_nope;
-  int64_t qn_st, qn_sh;
-  const uint16_t* q_pe;
-  int64_t qp_st, qp_sh;
-  const uint16_t* kv_c;
-  int64_t kv_st;
-  const uint16_t* k_pe;
-  int64_t kp_st;
-  const int64_t* slots;
-  const int32_t* positions;
-  const float* cos_sin;
-  int64_t rope_rows;
-  const float* q_scale;
-  const float* kv_scale;
-  int64_t T;
-  int64_t H;
-  uint64_t h_magic;  // ceil(2^64 / H) for H >= 2, see div_heads
-  int64_t cache_rows;
-  int64_t rows;  // T * (H + 1)
-  uint8_t* q_out;
-  uint8_t* cache;
-  int32_t* status;
-};
-
-// q / H for 0 <= q < 2^31 by one multiply-high: with M = ceil(2^64 / H),
-// floor(q M / 2^64) = floor(q / H + q (M - 2^64/H) / 2^64), and the added term
-// is below 2^-33 while the fractional part of q / H is at most 1 - 2^-16.
-__device__ __forceinline__ int64_t div_heads(const Args& a, int64_t q) {
-  return a.H == 1 ? q : static_cast<int64_t>(__umul64hi(static_cast<uint64_t>(q), a.h_magic));
-}
-
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-__device__ __forceinline__ void report(int32_t* status, int32_t bit) {
-  if (status != nullptr) atomicOr(status, bit);
-}
-
-// Rotation of pair `i` for token t: (cos, sin) from the table row of its position.
-struct Rot {
-  float c, s;
-  bool on;
-};
-
-__device__ __forceinline__ Rot load_rotation(const Args& a, int64_t t, int i) {
-  Rot r{1.0f, 0.0f, false};
-  const int64_t pos = __ldg(a.positions + t);
-  if (pos >= 0 && pos < a.rope_rows) {
-    const float* row = a.cos_sin + pos * kPe;
-    r.c = __ldg(row + i);
-    r.s = __ldg(row + kHalfPe + i);
-    r.on = true;
-  }
-  return r;
-}
+constexpr int kSmallMaxThreads = 1024;
+constexpr int kSmallMaxRowsPerBlock = 15;  // 68 * 15 = 1020 threads
+constexpr int kTokenLanesPerRow = 36;      // 32 nope threads (two chunks each) + 4 pe threads
+constexpr int kTokenMaxRowsPerBlock = kSmallMaxThreads / kTokenLanesPerRow;  // 28
 
 // Nope chunk `chunk` (8 values) of a row: 16 bytes in, 16 (bf16) or 8 (e4m3) out.
 template <bool FP8, bool FAST>
@@ -120,219 +57,234 @@ __device__ __forceinline__ void store_nope(uint8_t* dst, int chunk, const uint4 
   }
 }
 
-// RoPE pair i of a row: pe[i] in the low half of `pe`, pe[i+32] in the high half.
-template <bool FP8, bool ROPE, bool FAST>
-__device__ __forceinline__ void store_pe(uint8_t* dst, int i, uint32_t pe, const Rot& r, const Divisor& d) {
-  float a = bf16_lo(pe);
-  float b = bf16_hi(pe);
-  bool rotated = false;
+// Rotation of the pairs 8j .. 8j+7 of token t: cos and sin from the table row
+// of its position, or `on` false when RoPE is off or the position is out of
+// range.
+struct Rot8 {
+  float c[8], s[8];
+  bool on;
+};
+
+template <bool ROPE>
+__device__ __forceinline__ Rot8 load_rot8(const Args& a, int64_t t, int j) {
+  Rot8 r;
+  r.on = false;
   if constexpr (ROPE) {
-    if (r.on) {
-      float ya, yb;
-      rope_pair(a, b, r.c, r.s, ya, yb);
-      a = ya;
-      b = yb;
-      rotated = true;
+    const int64_t pos = __ldg(a.positions + t);
+    if (pos >= 0 && pos < a.rope_rows) {
+      const float* row = a.cos_sin + pos * kPe + 8 * j;
+      if (a.tab_vec) {
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(row));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(row) + 1);
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(row + kHalfPe));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(row + kHalfPe) + 1);
+        r.c[0] = c0.x; r.c[1] = c0.y; r.c[2] = c0.z; r.c[3] = c0.w;
+        r.c[4] = c1.x; r.c[5] = c1.y; r.c[6] = c1.z; r.c[7] = c1.w;
+        r.s[0] = s0.x; r.s[1] = s0.y; r.s[2] = s0.z; r.s[3] = s0.w;
+        r.s[4] = s1.x; r.s[5] = s1.y; r.s[6] = s1.z; r.s[7] = s1.w;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          r.c[k] = __ldg(row + k);
+          r.s[k] = __ldg(row + kHalfPe + k);
+        }
+      }
+      r.on = true;
     }
   }
+  return r;
+}
+
+// pe values 8j .. 8j+7 (`lo`) and 32+8j .. 32+8j+7 (`hi`) of one row as bf16
+// words (value 2k in the low half of word k): two 16-byte loads when the row
+// is 16-byte aligned, else sixteen 2-byte loads.
+__device__ __forceinline__ void load_pe8(const uint16_t* pe, int j, bool vec, uint4& lo, uint4& hi) {
+  if (vec) {
+    lo = ld_cg16(pe + 8 * j);
+    hi = ld_cg16(pe + kHalfPe + 8 * j);
+  } else {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      w[k] = static_cast<uint32_t>(__ldcg(pe + 8 * j + 2 * k)) |
+             (static_cast<uint32_t>(__ldcg(pe + 8 * j + 2 * k + 1)) << 16);
+      w[4 + k] = static_cast<uint32_t>(__ldcg(pe + kHalfPe + 8 * j + 2 * k)) |
+                 (static_cast<uint32_t>(__ldcg(pe + kHalfPe + 8 * j + 2 * k + 1)) << 16);
+    }
+    lo = make_uint4(w[0], w[1], w[2], w[3]);
+    hi = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// The 8 RoPE pairs (8j + k, 32 + 8j + k), k < 8, of a row: rotate in fp32, encode,
+// store 2 x 16 bytes (bf16) or 2 x 8 bytes (e4m3).
+template <bool FP8, bool ROPE, bool FAST>
+__device__ __forceinline__ void store_pe8(uint8_t* row, int j, const uint4 lo, const uint4 hi, const Rot8& r,
+                                          const Divisor& d) {
+  const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
+  const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
+  float ya[8], yb[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float a = (k & 1) ? bf16_hi(wl[k >> 1]) : bf16_lo(wl[k >> 1]);
+    const float b = (k & 1) ? bf16_hi(wh[k >> 1]) : bf16_lo(wh[k >> 1]);
+    ya[k] = a;
+    yb[k] = b;
+    if (ROPE && r.on) rope_pair(a, b, r.c[k], r.s[k], ya[k], yb[k]);
+  }
   if constexpr (FP8) {
-    const uint32_t p = e4m3x2_of_f32<FAST>(a, b, d);
-    dst[kNope + i] = static_cast<uint8_t>(p & 0xffu);
-    dst[kNope + kHalfPe + i] = static_cast<uint8_t>((p >> 8) & 0xffu);
+    uint2 oa, ob;
+    oa.x = e4m3x2_of_f32<FAST>(ya[0], ya[1], d) | (e4m3x2_of_f32<FAST>(ya[2], ya[3], d) << 16);
+    oa.y = e4m3x2_of_f32<FAST>(ya[4], ya[5], d) | (e4m3x2_of_f32<FAST>(ya[6], ya[7], d) << 16);
+    ob.x = e4m3x2_of_f32<FAST>(yb[0], yb[1], d) | (e4m3x2_of_f32<FAST>(yb[2], yb[3], d) << 16);
+    ob.y = e4m3x2_of_f32<FAST>(yb[4], yb[5], d) | (e4m3x2_of_f32<FAST>(yb[6], yb[7], d) << 16);
+    *reinterpret_cast<uint2*>(row + kNope + 8 * j) = oa;
+    *reinterpret_cast<uint2*>(row + kNope + kHalfPe + 8 * j) = ob;
   } else {
-    const uint32_t p = rotated ? pack_bf16x2(a, b) : pe;  // unrotated: the input bits
-    uint16_t* o = reinterpret_cast<uint16_t*>(dst);
-    o[kNope + i] = static_cast<uint16_t>(p & 0xffffu);
-    o[kNope + kHalfPe + i] = static_cast<uint16_t>(p >> 16);
+    uint4 oa = lo, ob = hi;  // unrotated values keep their bits (NaN payloads included)
+    if (ROPE && r.on) {
+      oa = make_uint4(pack_bf16x2(ya[0], ya[1]), pack_bf16x2(ya[2], ya[3]), pack_bf16x2(ya[4], ya[5]),
+                      pack_bf16x2(ya[6], ya[7]));
+      ob = make_uint4(pack_bf16x2(yb[0], yb[1]), pack_bf16x2(yb[2], yb[3]), pack_bf16x2(yb[4], yb[5]),
+                      pack_bf16x2(yb[6], yb[7]));
+    }
+    *reinterpret_cast<uint4*>(row + 2 * (kNope + 8 * j)) = oa;
+    *reinterpret_cast<uint4*>(row + 2 * (kNope + kHalfPe + 8 * j)) = ob;
   }
 }
 
-__device__ __forceinline__ uint4 ld_chunk(const uint16_t* row, int chunk) {
-  return __ldcg(reinterpret_cast<const uint4*>(row) + chunk);
-}
-
-__device__ __forceinline__ uint32_t ld_pair(const uint16_t* pe, int i) {
-  return static_cast<uint32_t>(__ldcg(pe + i)) | (static_cast<uint32_t>(__ldcg(pe + kHalfPe + i)) << 16);
-}
-
 // ------------------------------------------------------------------------------------
-// split kernel: three warps per row
+// small-batch kernels (SPLIT: NC = 1, TOKEN: NC = 2 nope chunks per thread)
 // ------------------------------------------------------------------------------------
 
-template <bool FP8, bool ROPE, bool FAST>
-__device__ __forceinline__ void split_query_row(const Args& a, int64_t q, int part, int lane, const Divisor& d) {
-  const int64_t t = div_heads(a, q);
-  const int64_t h = q - t * a.H;
-  uint8_t* dst = a.q_out + q * (FP8 ? kRow : 2 * kRow);
-  if (part < 2) {
-    const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh;
-    const int chunk = part * 32 + lane;
-    pdl_wait();
-    const uint4 v = ld_chunk(src, chunk);
-    store_nope<FP8, FAST>(dst, chunk, v, d);
-  } else {
-    const uint16_t* src = a.q_pe + t * a.qp_st + h * a.qp_sh;
-    Rot r{1.0f, 0.0f, false};
-    if constexpr (ROPE) r = load_rotation(a, t, lane);
-    pdl_wait();
-    const uint32_t pe = ld_pair(src, lane);
-    store_pe<FP8, ROPE, FAST>(dst, lane, pe, r, d);
-  }
-}
-
-template <bool FP8, bool ROPE, bool FAST>
-__device__ __forceinline__ void split_cache_row(const Args& a, int64_t t, int part, int lane, const Divisor& d) {
+template <int NC, bool FP8, bool ROPE, bool FAST>
+__device__ __forceinline__ void small_cache_row(const Args& a, int64_t t, bool pe, int part, const Divisor& d) {
+  constexpr int kNopeLanes = 64 / NC;
   const int64_t slot = __ldg(a.slots + t);
   const bool in_range = slot >= 0 && slot < a.cache_rows;
   uint8_t* dst = a.cache + (in_range ? slot : 0) * (FP8 ? kRow : 2 * kRow);
-  if (part < 2) {
-    const int chunk = part * 32 + lane;
-    const uint4 v = ld_chunk(a.kv_c + t * a.kv_st, chunk);
-    if (part == 0 && lane == 0 && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
-    if (in_range) store_nope<FP8, FAST>(dst, chunk, v, d);
-  } else {
-    Rot r{1.0f, 0.0f, false};
-    if constexpr (ROPE) {
-      r = load_rotation(a, t, lane);
-      if (lane == 0 && !r.on) report(a.status, MLA_STATUS_POS_RANGE);
+  if (!pe) {
+    const uint16_t* src = a.kv_c + t * a.kv_st;
+    uint4 v[NC];
+#pragma unroll
+    for (int k = 0; k < NC; ++k) v[k] = ld_cg16(src + 8 * (part + k * kNopeLanes));
+    if (part == 0 && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
+    if (in_range) {
+#pragma unroll
+      for (int k = 0; k < NC; ++k) store_nope<FP8, FAST>(dst, part + k * kNopeLanes, v[k], d);
     }
-    const uint32_t pe = ld_pair(a.k_pe + t * a.kp_st, lane);
-    if (in_range) store_pe<FP8, ROPE, FAST>(dst, lane, pe, r, d);
+  } else {
+    const Rot8 rot = load_rot8<ROPE>(a, t, part);
+    if (ROPE && part == 0 && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
+    uint4 lo, hi;
+    load_pe8(a.k_pe + t * a.kp_st, part, a.kpe_vec != 0, lo, hi);
+    if (in_range) store_pe8<FP8, ROPE, FAST>(dst, part, lo, hi, rot, d);
   }
 }
 
-template <bool QF8, bool KVF8, bool ROPE>
-__global__ void __launch_bounds__(kSplitThreadsPerRow * kSplitMaxRowsPerBlock) mla_epilogue_split_kernel(const Args a) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int rows_per_block = blockDim.x / kSplitThreadsPerRow;
-  const int64_t g = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp / 3;
-  const int part = warp % 3;
+template <int NC, bool FP8, bool ROPE, bool FAST>
+__device__ __forceinline__ void small_query_row(const Args& a, int64_t q, bool pe, int part, const Divisor& d) {
+  constexpr int kNopeLanes = 64 / NC;
+  const int64_t t = div_heads(a, q);
+  const int64_t h = q - t * a.H;
+  uint8_t* dst = a.q_out + q * (FP8 ? kRow : 2 * kRow);
+  if (!pe) {
+    const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh;
+    pdl_wait();
+    uint4 v[NC];
+#pragma unroll
+    for (int k = 0; k < NC; ++k) v[k] = ld_cg16(src + 8 * (part + k * kNopeLanes));
+#pragma unroll
+    for (int k = 0; k < NC; ++k) store_nope<FP8, FAST>(dst, part + k * kNopeLanes, v[k], d);
+  } else {
+    const uint16_t* src = a.q_pe + t * a.qp_st + h * a.qp_sh;
+    const Rot8 rot = load_rot8<ROPE>(a, t, part);
+    pdl_wait();
+    uint4 lo, hi;
+    load_pe8(src, part, a.qpe_vec != 0, lo, hi);
+    store_pe8<FP8, ROPE, FAST>(dst, part, lo, hi, rot, d);
+  }
+}
+
+template <int NC, bool QF8, bool KVF8, bool ROPE>
+__global__ void __launch_bounds__(kSmallMaxThreads) mla_epilogue_small_kernel(const Args a) {
+  constexpr int kNopeLanes = 64 / NC;
+  const int R = a.rows_per_block;
+  const int tid = static_cast<int>(threadIdx.x);
+  const int nope_threads = kNopeLanes * R;
+  const bool pe = tid >= nope_threads;
+  const int u = pe ? tid - nope_threads : tid;
+  const int r = pe ? (u >> 2) : (u / kNopeLanes);
+  const int part = pe ? (u & 3) : (u % kNopeLanes);
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * R + r;
   if (g < a.rows) {
-    // the row's divisor (scales are read before any wait); quotients take the
-    // corrected-reciprocal path unless the scale is outside [2^-64, 2^64]
+    // the divisor of the row's scale (read before any wait); quotients take
+    // the corrected-reciprocal path unless the scale is outside [2^-64, 2^64]
     if (g < a.T) {
-      Divisor d{};
-      d.fast = true;
-      if constexpr (KVF8) d = make_divisor(__ldg(a.kv_scale));
+      const Divisor d = divisor_of<KVF8>(a.kv_scale);
       if (d.fast) {
-        split_cache_row<KVF8, ROPE, true>(a, g, part, lane, d);
+        small_cache_row<NC, KVF8, ROPE, true>(a, g, pe, part, d);
       } else {
-        split_cache_row<KVF8, ROPE, false>(a, g, part, lane, d);
+        small_cache_row<NC, KVF8, ROPE, false>(a, g, pe, part, d);
       }
     } else {
-      Divisor d{};
-      d.fast = true;
-      if constexpr (QF8) d = make_divisor(__ldg(a.q_scale));
+      const Divisor d = divisor_of<QF8>(a.q_scale);
       if (d.fast) {
-        split_query_row<QF8, ROPE, true>(a, g - a.T, part, lane, d);
+        small_query_row<NC, QF8, ROPE, true>(a, g - a.T, pe, part, d);
       } else {
-        split_query_row<QF8, ROPE, false>(a, g - a.T, part, lane, d);
+        small_query_row<NC, QF8, ROPE, false>(a, g - a.T, pe, part, d);
       }
     }
-  }
-  pdl_trigger();
-}
-
-// ------------------------------------------------------------------------------------
-// rows kernel: one warp per row, grid-stride over rows
-// ------------------------------------------------------------------------------------
-
-template <bool QF8, bool KVF8, bool ROPE, bool FAST>
-__device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, const Divisor& dk) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int64_t wid = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  bool waited = false;
-
-  for (int64_t g = wid; g < a.rows; g += warps) {
-    // 1. addresses, slot and rotation: nothing here depends on the upstream kernel
-    const bool is_cache = g < a.T;
-    int64_t t;
-    const uint16_t* nope;
-    const uint16_t* pe;
-    uint8_t* dst = nullptr;
-    if (is_cache) {
-      t = g;
-      nope = a.kv_c + t * a.kv_st;
-      pe = a.k_pe + t * a.kp_st;
-      const int64_t slot = __ldg(a.slots + t);
-      if (slot >= 0 && slot < a.cache_rows) {
-        dst = a.cache + slot * (KVF8 ? kRow : 2 * kRow);
-      } else if (slot >= a.cache_rows && lane == 0) {
-        report(a.status, MLA_STATUS_SLOT_RANGE);
-      }
-    } else {
-      const int64_t q = g - a.T;
-      t = div_heads(a, q);
-      const int64_t h = q - t * a.H;
-      nope = a.q_nope + t * a.qn_st + h * a.qn_sh;
-      pe = a.q_pe + t * a.qp_st + h * a.qp_sh;
-      dst = a.q_out + q * (QF8 ? kRow : 2 * kRow);
-    }
-    Rot rot{1.0f, 0.0f, false};
-    if constexpr (ROPE) {
-      rot = load_rotation(a, t, lane);
-      if (is_cache && lane == 0 && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
-    }
-
-    // 2. query rows read what the upstream kernel wrote: wait for it once
-    if (!is_cache && !waited) {
-      pdl_wait();
-      waited = true;
-    }
-
-    // 3. the row's loads, then 4. convert and store
-    const uint4 n0 = ld_chunk(nope, lane);
-    const uint4 n1 = ld_chunk(nope, lane + 32);
-    const uint32_t p = ld_pair(pe, lane);
-    if (dst == nullptr) continue;
-    if (is_cache) {
-      store_nope<KVF8, FAST>(dst, lane, n0, dk);
-      store_nope<KVF8, FAST>(dst, lane + 32, n1, dk);
-      store_pe<KVF8, ROPE, FAST>(dst, lane, p, rot, dk);
-    } else {
-      store_nope<QF8, FAST>(dst, lane, n0, dq);
-      store_nope<QF8, FAST>(dst, lane + 32, n1, dq);
-      store_pe<QF8, ROPE, FAST>(dst, lane, p, rot, dq);
-    }
-  }
-}
-
-template <bool QF8, bool KVF8, bool ROPE>
-__global__ void __launch_bounds__(256, rows_blocks_per_sm(QF8, KVF8)) mla_epilogue_rows_kernel(const Args a) {
-  // scales are read before any wait; the whole body takes the corrected-
-  // reciprocal quotient unless a scale is outside [2^-64, 2^64]
-  Divisor dq{}, dk{};
-  dq.fast = dk.fast = true;
-  if constexpr (QF8) dq = make_divisor(__ldg(a.q_scale));
-  if constexpr (KVF8) dk = make_divisor(__ldg(a.kv_scale));
-  if (dq.fast && dk.fast) {
-    rows_body<QF8, KVF8, ROPE, true>(a, dq, dk);
-  } else {
-    rows_body<QF8, KVF8, ROPE, false>(a, dq, dk);
   }
   pdl_trigger();
 }
 
 // kernel tables indexed by (ROPE, Q_FP8, KV_FP8) = flags & 7
-template <int F>
-const void* split_kernel_for() {
-  return reinterpret_cast<const void*>(
-      &mla_epilogue_split_kernel<(F & MLA_FLAG_Q_FP8) != 0, (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
-}
-template <int F>
-const void* rows_kernel_for() {
-  return reinterpret_cast<const void*>(
-      &mla_epilogue_rows_kernel<(F & MLA_FLAG_Q_FP8) != 0, (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
+template <int NC, int F>
+const void* small_kernel_for() {
+  return reinterpret_cast<const void*>(&mla_epilogue_small_kernel<NC, (F & MLA_FLAG_Q_FP8) != 0,
+                                                                  (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
 }
 
-const void* const kSplitKernels[8] = {split_kernel_for<0>(), split_kernel_for<1>(), split_kernel_for<2>(),
-                                      split_kernel_for<3>(), split_kernel_for<4>(), split_kernel_for<5>(),
-                                      split_kernel_for<6>(), split_kernel_for<7>()};
-const void* const kRowsKernels[8] = {rows_kernel_for<0>(), rows_kernel_for<1>(), rows_kernel_for<2>(),
-                                     rows_kernel_for<3>(), rows_kernel_for<4>(), rows_kernel_for<5>(),
-                                     rows_kernel_for<6>(), rows_kernel_for<7>()};
+const void* const kSplitKernels[8] = {small_kernel_for<1, 0>(), small_kernel_for<1, 1>(), small_kernel_for<1, 2>(),
+                                      small_kernel_for<1, 3>(), small_kernel_for<1, 4>(), small_kernel_for<1, 5>(),
+                                      small_kernel_for<1, 6>(), small_kernel_for<1, 7>()};
+const void* const kTokenKernels[8] = {small_kernel_for<2, 0>(), small_kernel_for<2, 1>(), small_kernel_for<2, 2>(),
+                                      small_kernel_for<2, 3>(), small_kernel_for<2, 4>(), small_kernel_for<2, 5>(),
+                                      small_kernel_for<2, 6>(), small_kernel_for<2, 7>()};
+
+// ------------------------------------------------------------------------------------
+// host helpers shared by every launcher (mla_runtime.h)
+// ------------------------------------------------------------------------------------
+
+namespace {
+thread_local int32_t g_last_cuda_error = 0;
+std::atomic<int32_t> g_sm_count[kMaxDevices];
+}  // namespace
+
+mla_status cuda_failure(cudaError_t e) {
+  g_last_cuda_error = static_cast<int32_t>(e);
+  (void)cudaGetLastError();
+  return MLA_ERR_CUDA;
+}
+
+mla_status current_device(int* dev_out, int32_t* sm_count) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess && (dev < 0 || dev >= kMaxDevices)) e = cudaErrorInvalidDevice;
+  if (e != cudaSuccess) return cuda_failure(e);
+  int32_t n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    int v = 0;
+    e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_failure(e);
+    n = v;
+    g_sm_count[dev].store(n, std::memory_order_relaxed);
+  }
+  if (dev_out != nullptr) *dev_out = dev;
+  *sm_count = n;
+  return MLA_OK;
+}
 
 }  // namespace mla
 
@@ -343,56 +295,48 @@ const void* const kRowsKernels[8] = {rows_kernel_for<0>(), rows_kernel_for<1>(),
 namespace {
 
 constexpr uint32_t kKnownFlags = MLA_FLAG_ROPE | MLA_FLAG_Q_FP8 | MLA_FLAG_KV_FP8 | MLA_FLAG_PDL |
-                                 MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS;
-constexpr int kMaxDevices = 64;
+                                 MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS | MLA_FLAG_FORCE_TOKEN;
+constexpr uint32_t kForceFlags = MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS | MLA_FLAG_FORCE_TOKEN;
 
-mla_tuning g_tuning = {4608, 2, 8, mla::kRowsMaxBlocksPerSm};
-int g_sm_count[kMaxDevices] = {0};
-thread_local int32_t g_last_cuda_error = 0;
+mla_tuning g_tuning = {4608, 8, mla::kRowsDefaultWarps, mla::kRowsMaxBlocksPerSm};
 
 bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
 
-mla_status device_sm_count(int32_t* out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess && (dev < 0 || dev >= kMaxDevices)) e = cudaErrorInvalidDevice;
-  if (e == cudaSuccess && g_sm_count[dev] <= 0) {
-    int n = 0;
-    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) g_sm_count[dev] = n;
-  }
-  if (e != cudaSuccess) {
-    g_last_cuda_error = static_cast<int32_t>(e);
-    (void)cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
-  *out = g_sm_count[dev];
-  return MLA_OK;
+bool one_force_flag(uint32_t flags) {
+  const uint32_t f = flags & kForceFlags;
+  return (f & (f - 1)) == 0;
 }
 
 mla_status make_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla_plan* p) {
   const int64_t rows = T * (H + 1);
-  const bool split = (flags & MLA_FLAG_FORCE_SPLIT) ? true
-                     : (flags & MLA_FLAG_FORCE_ROWS) ? false
-                                                      : (rows <= g_tuning.split_max_rows);
+  int32_t mode;
+  if (flags & MLA_FLAG_FORCE_SPLIT) {
+    mode = MLA_MODE_SPLIT;
+  } else if (flags & MLA_FLAG_FORCE_ROWS) {
+    mode = MLA_MODE_ROWS;
+  } else if (flags & MLA_FLAG_FORCE_TOKEN) {
+    mode = MLA_MODE_TOKEN;
+  } else if (T == 1) {
+    mode = MLA_MODE_TOKEN;
+  } else {
+    mode = rows <= g_tuning.split_max_rows ? MLA_MODE_SPLIT : MLA_MODE_ROWS;
+  }
+  p->mode = mode;
   p->sm_count = sm_count;
-  if (split) {
+  if (mode == MLA_MODE_SPLIT) {
     const int32_t rpb = g_tuning.split_rows_per_block;
-    p->mode = MLA_MODE_SPLIT;
     p->rows_per_block = rpb;
-    p->threads_per_block = mla::kSplitThreadsPerRow * rpb;
+    p->threads_per_block = (64 + 4) * rpb;
+    p->blocks = (rows + rpb - 1) / rpb;
+  } else if (mode == MLA_MODE_TOKEN) {
+    // all rows of one token in one block where they fit
+    const int64_t rpb = H + 1 < mla::kTokenMaxRowsPerBlock ? H + 1 : mla::kTokenMaxRowsPerBlock;
+    p->rows_per_block = static_cast<int32_t>(rpb);
+    p->threads_per_block = mla::kTokenLanesPerRow * static_cast<int32_t>(rpb);
     p->blocks = (rows + rpb - 1) / rpb;
   } else {
-    const int32_t w = g_tuning.rows_warps_per_block;
-    const int64_t per_block = w;
-    const int64_t need = (rows + per_block - 1) / per_block;
-    const int32_t resident = mla::rows_blocks_per_sm((flags & MLA_FLAG_Q_FP8) != 0, (flags & MLA_FLAG_KV_FP8) != 0);
-    const int32_t per_sm = g_tuning.rows_blocks_per_sm < resident ? g_tuning.rows_blocks_per_sm : resident;
-    const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
-    p->mode = MLA_MODE_ROWS;
-    p->rows_per_block = 1;
-    p->threads_per_block = 32 * w;
-    p->blocks = need < cap ? need : cap;
+    mla::rows_plan(rows, (flags & MLA_FLAG_Q_FP8) != 0, (flags & MLA_FLAG_KV_FP8) != 0, sm_count,
+                   g_tuning.rows_blocks_per_sm, g_tuning.rows_warps_per_block, p);
   }
   return MLA_OK;
 }
@@ -407,20 +351,22 @@ const char* mla_status_string(mla_status s) {
     case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: null pointer, bad size or stride, or conflicting flags";
     case MLA_ERR_ALIGNMENT: return "MLA_ERR_ALIGNMENT: a pointer or stride breaks the 16-byte row rule";
     case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: unknown flag bit";
-    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: the CUDA runtime refused the launch";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: the CUDA runtime refused the call";
   }
   return "unknown mla_status";
 }
 
-int32_t mla_last_cuda_error(void) { return g_last_cuda_error; }
+int32_t mla_last_cuda_error(void) { return mla::g_last_cuda_error; }
 
 void mla_epilogue_set_tuning(const mla_tuning* t) {
   if (t == nullptr) return;
   if (t->split_max_rows > 0) g_tuning.split_max_rows = t->split_max_rows;
   if (t->split_rows_per_block > 0)
-    g_tuning.split_rows_per_block = t->split_rows_per_block < mla::kSplitMaxRowsPerBlock ? t->split_rows_per_block
-                                                                                          : mla::kSplitMaxRowsPerBlock;
-  if (t->rows_warps_per_block > 0) g_tuning.rows_warps_per_block = t->rows_warps_per_block < 8 ? t->rows_warps_per_block : 8;
+    g_tuning.split_rows_per_block =
+        t->split_rows_per_block < mla::kSmallMaxRowsPerBlock ? t->split_rows_per_block : mla::kSmallMaxRowsPerBlock;
+  if (t->rows_warps_per_block > 0)
+    g_tuning.rows_warps_per_block =
+        t->rows_warps_per_block < mla::kRowsMaxConsumerWarps ? t->rows_warps_per_block : mla::kRowsMaxConsumerWarps;
   if (t->rows_blocks_per_sm > 0)
     g_tuning.rows_blocks_per_sm =
         t->rows_blocks_per_sm < mla::kRowsMaxBlocksPerSm ? t->rows_blocks_per_sm : mla::kRowsMaxBlocksPerSm;
@@ -432,10 +378,10 @@ void mla_epilogue_get_tuning(mla_tuning* out) {
 
 mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla_plan* out) {
   if (out == nullptr || T < 1 || H < 1 || H > 65536) return MLA_ERR_INVALID_ARG;
-  if ((flags & MLA_FLAG_FORCE_SPLIT) && (flags & MLA_FLAG_FORCE_ROWS)) return MLA_ERR_INVALID_ARG;
+  if (!one_force_flag(flags)) return MLA_ERR_INVALID_ARG;
   if (T > (static_cast<int64_t>(INT_MAX)) / (H + 1)) return MLA_ERR_INVALID_ARG;
   if (sm_count <= 0) {
-    const mla_status s = device_sm_count(&sm_count);
+    const mla_status s = mla::current_device(nullptr, &sm_count);
     if (s != MLA_OK) return s;
   }
   return make_plan(T, H, flags, sm_count, out);
@@ -453,7 +399,7 @@ mla_status mla_epilogue_launch(
     uint32_t flags, void* q_out, void* cache, int32_t* status, mla_stream_t stream) {
   // ---- scalars and flags
   if ((flags & ~kKnownFlags) != 0) return MLA_ERR_UNSUPPORTED;
-  if ((flags & MLA_FLAG_FORCE_SPLIT) && (flags & MLA_FLAG_FORCE_ROWS)) return MLA_ERR_INVALID_ARG;
+  if (!one_force_flag(flags)) return MLA_ERR_INVALID_ARG;
   if (T < 0 || H < 1 || H > 65536 || block_size < 1 || num_blocks < 0) return MLA_ERR_INVALID_ARG;
   if (T > static_cast<int64_t>(INT_MAX) / (H + 1)) return MLA_ERR_INVALID_ARG;
   if (num_blocks > (INT64_C(1) << 50) / block_size) return MLA_ERR_INVALID_ARG;
@@ -487,7 +433,7 @@ mla_status mla_epilogue_launch(
 
   // ---- plan and launch
   int32_t sms = 0;
-  mla_status s = device_sm_count(&sms);
+  mla_status s = mla::current_device(nullptr, &sms);
   if (s != MLA_OK) return s;
   mla_plan plan;
   s = make_plan(T, H, flags, sms, &plan);
@@ -518,14 +464,27 @@ mla_status mla_epilogue_launch(
   a.q_out = static_cast<uint8_t*>(q_out);
   a.cache = static_cast<uint8_t*>(cache);
   a.status = status;
+  a.rows_per_block = plan.rows_per_block;
+  a.qpe_vec = aligned(q_pe, 16) && (T == 1 || q_pe_stride_t % 8 == 0) && (H == 1 || q_pe_stride_h % 8 == 0);
+  a.kpe_vec = aligned(k_pe, 16) && (T == 1 || k_pe_stride_t % 8 == 0);
+  a.tab_vec = rope && aligned(cos_sin, 16);
 
   const int k = static_cast<int>(flags & 7u);
-  const void* fn = (plan.mode == MLA_MODE_SPLIT) ? mla::kSplitKernels[k] : mla::kRowsKernels[k];
+  const void* fn = nullptr;
+  size_t smem = 0;
+  if (plan.mode == MLA_MODE_SPLIT) {
+    fn = mla::kSplitKernels[k];
+  } else if (plan.mode == MLA_MODE_TOKEN) {
+    fn = mla::kTokenKernels[k];
+  } else {
+    s = mla::rows_kernel(k, &fn, &smem);
+    if (s != MLA_OK) return s;
+  }
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.blocks), 1, 1);
   cfg.blockDim = dim3(static_cast<unsigned>(plan.threads_per_block), 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   if (flags & MLA_FLAG_PDL) {
@@ -536,11 +495,7 @@ mla_status mla_epilogue_launch(
   }
   void* args[] = {&a};
   const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
-  if (e != cudaSuccess) {
-    g_last_cuda_error = static_cast<int32_t>(e);
-    (void)cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
+  if (e != cudaSuccess) return mla::cuda_failure(e);
   return MLA_OK;
 }
 

@@ -7,6 +7,7 @@
 
 #include "latent_math.cuh"
 #include "mla_harness.h"
+#include "mla_runtime.h"
 
 namespace mla {
 namespace harness {
@@ -39,6 +40,8 @@ __global__ void __launch_bounds__(256) produce_kernel(const uint4* __restrict__ 
 }
 
 __global__ void empty_kernel() {}
+
+__global__ void empty_wait_kernel() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Quotient of one fp32 through the epilogue's e4m3 path (the pair function
 // with the second lane unused), returned as the fp32 quotient it encodes.
@@ -124,13 +127,7 @@ __global__ void __launch_bounds__(256) consume_kernel(const uint8_t* q_out, cons
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-mla_status finish(cudaError_t e) {
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
-  return MLA_OK;
-}
+mla_status finish(cudaError_t e) { return e == cudaSuccess ? MLA_OK : cuda_failure(e); }
 
 mla_status launch(const void* fn, dim3 grid, dim3 block, bool pdl, cudaStream_t stream, void** args) {
   cudaLaunchConfig_t cfg = {};
@@ -165,9 +162,9 @@ mla_status mla_harness_produce(const void* src_nope, const void* src_pe, void* q
   if (!aligned16(src_nope) || !aligned16(src_pe) || !aligned16(q_nope) || !aligned16(q_pe) ||
       (q_nope_stride_t % 8) || (q_nope_stride_h % 8) || (q_pe_stride_t % 8) || (q_pe_stride_h % 8))
     return MLA_ERR_ALIGNMENT;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return finish(cudaErrorUnknown);
+  int32_t sms = 0;
+  const mla_status s = mla::current_device(nullptr, &sms);
+  if (s != MLA_OK) return s;
   const int64_t rows = T * H;
   int64_t blocks = (rows + 7) / 8;
   if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
@@ -182,9 +179,11 @@ mla_status mla_harness_produce(const void* src_nope, const void* src_pe, void* q
 
 mla_status mla_harness_empty(int64_t blocks, int32_t threads, uint32_t flags, mla_stream_t stream) {
   using namespace mla::harness;
-  if ((flags & ~MLA_FLAG_PDL) != 0) return MLA_ERR_UNSUPPORTED;
+  if ((flags & ~(MLA_FLAG_PDL | MLA_HARNESS_EMPTY_WAIT)) != 0) return MLA_ERR_UNSUPPORTED;
   if (blocks < 1 || blocks > INT32_MAX || threads < 1 || threads > 1024) return MLA_ERR_INVALID_ARG;
-  return launch(reinterpret_cast<const void*>(&empty_kernel), dim3(static_cast<unsigned>(blocks)),
+  const void* fn = (flags & MLA_HARNESS_EMPTY_WAIT) ? reinterpret_cast<const void*>(&empty_wait_kernel)
+                                                    : reinterpret_cast<const void*>(&empty_kernel);
+  return launch(fn, dim3(static_cast<unsigned>(blocks)),
                 dim3(static_cast<unsigned>(threads)), (flags & MLA_FLAG_PDL) != 0,
                 reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
@@ -199,8 +198,12 @@ mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t count, un
   if (e == cudaSuccess) e = cudaMemsetAsync(result + 2, 0xff, sizeof(unsigned long long), s);
   if (e != cudaSuccess) return finish(e);
   if (count == 0) return MLA_OK;
+  int32_t sms = 0;
+  const mla_status st = mla::current_device(nullptr, &sms);
+  if (st != MLA_OK) return st;
   void* args[] = {&scale, &first, &count, &result};
-  return launch(reinterpret_cast<const void*>(&div_check_kernel), dim3(148 * 16), dim3(256), false, s, args);
+  return launch(reinterpret_cast<const void*>(&div_check_kernel), dim3(static_cast<unsigned>(sms) * 16), dim3(256),
+                false, s, args);
 }
 
 mla_status mla_harness_consume(const void* q_out, const void* cache, const int64_t* slot_mapping, int64_t T,
@@ -213,9 +216,12 @@ mla_status mla_harness_consume(const void* q_out, const void* cache, const int64
   if (!aligned16(q_out) || (cache && !aligned16(cache)) || (reinterpret_cast<uintptr_t>(scores) & 3u) ||
       (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
     return MLA_ERR_ALIGNMENT;
+  int32_t sms = 0;
+  const mla_status s = mla::current_device(nullptr, &sms);
+  if (s != MLA_OK) return s;
   const int64_t rows = T * H;
   int64_t blocks = (rows + 7) / 8;
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
   const bool qf8 = (flags & MLA_FLAG_Q_FP8) != 0, kvf8 = (flags & MLA_FLAG_KV_FP8) != 0;
   const void* fn = qf8 ? (kvf8 ? reinterpret_cast<const void*>(&consume_kernel<true, true>)
                                : reinterpret_cast<const void*>(&consume_kernel<true, false>))

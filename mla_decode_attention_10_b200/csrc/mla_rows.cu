@@ -1,0 +1,195 @@
+// mla_rows.cu -- the large-batch (MLA_MODE_ROWS) kernel of the fused MLA
+// decode epilogue: one warp per row, grid-stride over rows, the grid a
+// multiple of the SM count sized to the kernel's register-limited residency
+// (lane l moves nope chunks l and l + 32 and rotates pe pair l).
+//
+// Rows [0, T) are cache rows and never wait; query rows execute
+// griddepcontrol.wait once, before their first read of q_nope / q_pe (vLLM
+// PR #54896 report, 实现拆解 item 2); every thread triggers its dependents
+// after its last store (评论区精华).
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "epilogue_device.cuh"
+#include "mla_rows.h"
+
+namespace mla {
+
+// Resident 256-thread blocks per SM the kernel is compiled for: 5 (a
+// 48-register cap) for bf16 outputs; 6 (40 registers) when an output is
+// e4m3, whose arithmetic leaves the kernel short of memory parallelism at 5.
+constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 6 : 5; }
+
+// Rotation of pair `i` for token t: (cos, sin) from the table row of its position.
+struct Rot {
+  float c, s;
+  bool on;
+};
+
+__device__ __forceinline__ Rot load_rotation(const Args& a, int64_t t, int i) {
+  Rot r{1.0f, 0.0f, false};
+  const int64_t pos = __ldg(a.positions + t);
+  if (pos >= 0 && pos < a.rope_rows) {
+    const float* row = a.cos_sin + pos * kPe;
+    r.c = __ldg(row + i);
+    r.s = __ldg(row + kHalfPe + i);
+    r.on = true;
+  }
+  return r;
+}
+
+template <bool FP8, bool FAST>
+__device__ __forceinline__ void store_nope(uint8_t* dst, int chunk, const uint4 v, const Divisor& d) {
+  if constexpr (FP8) {
+    *reinterpret_cast<uint2*>(dst + chunk * 8) = chunk_to_e4m3<FAST>(v, d);
+  } else {
+    *reinterpret_cast<uint4*>(dst + chunk * 16) = v;
+  }
+}
+
+// RoPE pair i of a row: pe[i] in the low half of `pe`, pe[i+32] in the high half.
+template <bool FP8, bool ROPE, bool FAST>
+__device__ __forceinline__ void store_pe(uint8_t* dst, int i, uint32_t pe, const Rot& r, const Divisor& d) {
+  float a = bf16_lo(pe);
+  float b = bf16_hi(pe);
+  bool rotated = false;
+  if constexpr (ROPE) {
+    if (r.on) {
+      float ya, yb;
+      rope_pair(a, b, r.c, r.s, ya, yb);
+      a = ya;
+      b = yb;
+      rotated = true;
+    }
+  }
+  if constexpr (FP8) {
+    const uint32_t p = e4m3x2_of_f32<FAST>(a, b, d);
+    dst[kNope + i] = static_cast<uint8_t>(p & 0xffu);
+    dst[kNope + kHalfPe + i] = static_cast<uint8_t>((p >> 8) & 0xffu);
+  } else {
+    const uint32_t p = rotated ? pack_bf16x2(a, b) : pe;  // unrotated: the input bits
+    uint16_t* o = reinterpret_cast<uint16_t*>(dst);
+    o[kNope + i] = static_cast<uint16_t>(p & 0xffffu);
+    o[kNope + kHalfPe + i] = static_cast<uint16_t>(p >> 16);
+  }
+}
+
+__device__ __forceinline__ uint4 ld_chunk(const uint16_t* row, int chunk) {
+  return __ldcg(reinterpret_cast<const uint4*>(row) + chunk);
+}
+
+__device__ __forceinline__ uint32_t ld_pair(const uint16_t* pe, int i) {
+  return static_cast<uint32_t>(__ldcg(pe + i)) | (static_cast<uint32_t>(__ldcg(pe + kHalfPe + i)) << 16);
+}
+
+// ------------------------------------------------------------------------------------
+// rows kernel: one warp per row, grid-stride over rows
+// ------------------------------------------------------------------------------------
+
+template <bool QF8, bool KVF8, bool ROPE, bool FAST>
+__device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, const Divisor& dk) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  bool waited = false;
+
+  for (int64_t g = wid; g < a.rows; g += warps) {
+    // 1. addresses, slot and rotation: nothing here depends on the upstream kernel
+    const bool is_cache = g < a.T;
+    int64_t t;
+    const uint16_t* nope;
+    const uint16_t* pe;
+    uint8_t* dst = nullptr;
+    if (is_cache) {
+      t = g;
+      nope = a.kv_c + t * a.kv_st;
+      pe = a.k_pe + t * a.kp_st;
+      const int64_t slot = __ldg(a.slots + t);
+      if (slot >= 0 && slot < a.cache_rows) {
+        dst = a.cache + slot * (KVF8 ? kRow : 2 * kRow);
+      } else if (slot >= a.cache_rows && lane == 0) {
+        report(a.status, MLA_STATUS_SLOT_RANGE);
+      }
+    } else {
+      const int64_t q = g - a.T;
+      t = div_heads(a, q);
+      const int64_t h = q - t * a.H;
+      nope = a.q_nope + t * a.qn_st + h * a.qn_sh;
+      pe = a.q_pe + t * a.qp_st + h * a.qp_sh;
+      dst = a.q_out + q * (QF8 ? kRow : 2 * kRow);
+    }
+    Rot rot{1.0f, 0.0f, false};
+    if constexpr (ROPE) {
+      rot = load_rotation(a, t, lane);
+      if (is_cache && lane == 0 && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
+    }
+
+    // 2. query rows read what the upstream kernel wrote: wait for it once
+    if (!is_cache && !waited) {
+      pdl_wait();
+      waited = true;
+    }
+
+    // 3. the row's loads, then 4. convert and store
+    const uint4 n0 = ld_chunk(nope, lane);
+    const uint4 n1 = ld_chunk(nope, lane + 32);
+    const uint32_t p = ld_pair(pe, lane);
+    if (dst == nullptr) continue;
+    if (is_cache) {
+      store_nope<KVF8, FAST>(dst, lane, n0, dk);
+      store_nope<KVF8, FAST>(dst, lane + 32, n1, dk);
+      store_pe<KVF8, ROPE, FAST>(dst, lane, p, rot, dk);
+    } else {
+      store_nope<QF8, FAST>(dst, lane, n0, dq);
+      store_nope<QF8, FAST>(dst, lane + 32, n1, dq);
+      store_pe<QF8, ROPE, FAST>(dst, lane, p, rot, dq);
+    }
+  }
+}
+
+template <bool QF8, bool KVF8, bool ROPE>
+__global__ void __launch_bounds__(256, rows_blocks_per_sm(QF8, KVF8)) mla_epilogue_rows_kernel(const Args a) {
+  // scales are read before any wait; the whole body takes the corrected-
+  // reciprocal quotient unless a scale is outside [2^-64, 2^64]
+  Divisor dq{}, dk{};
+  dq.fast = dk.fast = true;
+  if constexpr (QF8) dq = make_divisor(__ldg(a.q_scale));
+  if constexpr (KVF8) dk = make_divisor(__ldg(a.kv_scale));
+  if (dq.fast && dk.fast) {
+    rows_body<QF8, KVF8, ROPE, true>(a, dq, dk);
+  } else {
+    rows_body<QF8, KVF8, ROPE, false>(a, dq, dk);
+  }
+  pdl_trigger();
+}
+
+template <int F>
+const void* rows_kernel_for() {
+  return reinterpret_cast<const void*>(
+      &mla_epilogue_rows_kernel<(F & MLA_FLAG_Q_FP8) != 0, (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
+}
+
+const void* const kRowsKernels[8] = {rows_kernel_for<0>(), rows_kernel_for<1>(), rows_kernel_for<2>(),
+                                     rows_kernel_for<3>(), rows_kernel_for<4>(), rows_kernel_for<5>(),
+                                     rows_kernel_for<6>(), rows_kernel_for<7>()};
+
+void rows_plan(int64_t rows, bool qf8, bool kvf8, int32_t sm_count, int32_t blocks_per_sm, int32_t warps_per_block,
+               mla_plan* p) {
+  const int64_t need = (rows + warps_per_block - 1) / warps_per_block;
+  const int32_t resident = rows_blocks_per_sm(qf8, kvf8);
+  const int32_t per_sm = blocks_per_sm < resident ? blocks_per_sm : resident;
+  const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
+  p->mode = MLA_MODE_ROWS;
+  p->rows_per_block = 1;
+  p->threads_per_block = 32 * warps_per_block;
+  p->blocks = need < cap ? need : cap;
+}
+
+mla_status rows_kernel(int flag_bits, const void** fn, size_t* smem_bytes) {
+  *fn = kRowsKernels[flag_bits & 7];
+  *smem_bytes = 0;
+  return MLA_OK;
+}
+
+}  // namespace mla

@@ -31,6 +31,7 @@ MLA_FLAG_KV_FP8 = 4
 MLA_FLAG_PDL = 8
 MLA_FLAG_FORCE_SPLIT = 16
 MLA_FLAG_FORCE_ROWS = 32
+MLA_FLAG_FORCE_TOKEN = 64
 
 MLA_STATUS_SLOT_RANGE = 1
 MLA_STATUS_POS_RANGE = 2
@@ -38,6 +39,9 @@ MLA_STATUS_TIMEOUT = 4
 
 MLA_MODE_SPLIT = 1
 MLA_MODE_ROWS = 2
+MLA_MODE_TOKEN = 3
+
+MLA_HARNESS_EMPTY_WAIT = 256
 
 ROW = 576
 NOPE = 512

@@ -76,9 +76,10 @@ def _call(**kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(flags=64), E.MLA_ERR_UNSUPPORTED),
     (dict(flags=1 << 31), E.MLA_ERR_UNSUPPORTED),
+    (dict(flags=128), E.MLA_ERR_UNSUPPORTED),
     (dict(flags=E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=E.MLA_FLAG_FORCE_TOKEN | E.MLA_FLAG_FORCE_ROWS), E.MLA_ERR_INVALID_ARG),
     (dict(T=-1), E.MLA_ERR_INVALID_ARG),
     (dict(H=0), E.MLA_ERR_INVALID_ARG),
     (dict(H=65537), E.MLA_ERR_INVALID_ARG),
@@ -133,11 +134,13 @@ def test_size_one_dimensions_skip_stride_checks(lib):
 
 
 def test_plan_modes_and_grids(lib):
+    t = E.mla_epilogue_get_tuning()
     p = E.mla_epilogue_plan(64, 16, 0, sm_count=148)
-    assert p.mode == E.MLA_MODE_SPLIT and p.threads_per_block == 96 * p.rows_per_block
+    assert p.mode == E.MLA_MODE_SPLIT and p.threads_per_block == 68 * p.rows_per_block
+    assert p.rows_per_block == t.split_rows_per_block
     assert p.blocks == -(-64 * 17 // p.rows_per_block)
     # the default split threshold counts rows: 4608 = 271 tokens x 17 rows, rounded up
-    assert E.mla_epilogue_get_tuning().split_max_rows == 4608
+    assert t.split_max_rows == 4608
     assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
     assert E.mla_epilogue_plan(271, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
     assert E.mla_epilogue_plan(272, 16, 0, sm_count=148).mode == E.MLA_MODE_ROWS
@@ -145,17 +148,27 @@ def test_plan_modes_and_grids(lib):
     assert E.mla_epilogue_plan(36, 128, 0, sm_count=148).mode == E.MLA_MODE_ROWS
     p = E.mla_epilogue_plan(300, 16, 0, sm_count=148)
     assert p.mode == E.MLA_MODE_ROWS and p.threads_per_block % 32 == 0
-    assert p.blocks <= 148 * E.mla_epilogue_get_tuning().rows_blocks_per_sm
+    assert p.blocks <= 148 * t.rows_blocks_per_sm
     assert E.mla_epilogue_plan(1, 16, E.MLA_FLAG_FORCE_ROWS, sm_count=148).mode == E.MLA_MODE_ROWS
     assert E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148).mode == E.MLA_MODE_SPLIT
-    big = E.mla_epilogue_plan(8192, 16, 0, sm_count=148)
-    assert big.mode == E.MLA_MODE_ROWS and big.blocks == 148 * 5
-    big8 = E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_Q_FP8 | E.MLA_FLAG_KV_FP8, sm_count=148)
-    assert big8.mode == E.MLA_MODE_ROWS and big8.blocks == 148 * 6
+    assert E.mla_epilogue_plan(9, 16, E.MLA_FLAG_FORCE_TOKEN, sm_count=148).mode == E.MLA_MODE_TOKEN
     with pytest.raises(E.MlaError):
         E.mla_epilogue_plan(0, 16, 0, sm_count=148)
-    with pytest.raises(E.MlaError):
-        E.mla_epilogue_plan(4, 16, E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS, sm_count=148)
+    for bad in (E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS, E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_TOKEN,
+                E.MLA_FLAG_FORCE_ROWS | E.MLA_FLAG_FORCE_TOKEN):
+        with pytest.raises(E.MlaError):
+            E.mla_epilogue_plan(4, 16, bad, sm_count=148)
+
+
+@pytest.mark.parametrize("H,blocks", [(1, 1), (16, 1), (27, 1), (28, 2), (128, 5)])
+def test_single_token_plan_puts_the_token_in_one_block(lib, H, blocks):
+    """T == 1 takes MLA_MODE_TOKEN: 36 threads per row, every row of the
+    token in one block while H + 1 <= 28 rows fit in 1024 threads."""
+    p = E.mla_epilogue_plan(1, H, E.MLA_FLAG_ROPE, sm_count=148)
+    assert p.mode == E.MLA_MODE_TOKEN
+    assert p.rows_per_block == min(H + 1, 28) and p.threads_per_block == 36 * p.rows_per_block
+    assert p.blocks == blocks and p.blocks * p.rows_per_block >= H + 1
+    assert E.mla_epilogue_plan(2, H, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
 
 
 def test_tuning_moves_the_threshold_and_clamps(lib):
@@ -166,7 +179,11 @@ def test_tuning_moves_the_threshold_and_clamps(lib):
         assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_ROWS
         E.mla_epilogue_set_tuning(split_rows_per_block=99, rows_warps_per_block=99, rows_blocks_per_sm=99)
         t = E.mla_epilogue_get_tuning()
-        assert t.split_rows_per_block == 4 and t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 6
+        assert t.split_rows_per_block == 15 and 68 * t.split_rows_per_block <= 1024
+        assert t.rows_warps_per_block <= 16 and t.rows_blocks_per_sm <= 8
+        E.mla_epilogue_set_tuning(split_rows_per_block=3)
+        p = E.mla_epilogue_plan(5, 16, 0, sm_count=148)
+        assert p.rows_per_block == 3 and p.threads_per_block == 204 and p.blocks == 29
         E.mla_epilogue_set_tuning()  # all zero: unchanged
         assert E.mla_epilogue_get_tuning().split_max_rows == 64 * 17
     finally:
@@ -228,6 +245,29 @@ def test_absorb_validation(lib, kw, code):
     args.update(T=0, q_nope_c=None, w_uk=None, q_out=None)
     if code != E.MLA_ERR_UNSUPPORTED and kw.get("H", 1) >= 1 and kw.get("H", 1) < 65536 and kw.get("T", 0) >= 0:
         assert E.mla_absorb_launch(**args) == E.MLA_OK
+
+
+def test_cuda_failures_are_recorded_for_every_launcher(lib):
+    """A launcher that gets past its host checks and is refused by the CUDA
+    runtime returns MLA_ERR_CUDA and records the runtime's error code, which
+    mla_last_cuda_error() then reports (checked where no GPU is visible, so
+    the first runtime call fails)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a process without a visible GPU")
+    calls = {
+        "mla_absorb_launch": lambda: E.mla_absorb_launch(A, 16 * 128, 128, A, A, 16 * 64, 64, A, A, 8, A, 4, 16,
+                                                         E.MLA_FLAG_ROPE, A, None, None),
+        "mla_epilogue_launch": lambda: _call(),
+        "mla_epilogue_plan": lambda: E.lib().mla_epilogue_plan(4, 16, 0, 0, ctypes.byref(E.mla_plan())),
+        "mla_harness_produce": lambda: E.mla_harness_produce(A, A, A, 16 * 512, 512, A, 16 * 64, 64, 4, 16, 0, None),
+        "mla_harness_empty": lambda: E.mla_harness_empty(1, 32, 0, None),
+        "mla_harness_consume": lambda: E.mla_harness_consume(A, A, A, 4, 16, 64, 0, A, None),
+    }
+    for name, call in calls.items():
+        E.lib().mla_last_cuda_error.restype = ctypes.c_int32
+        assert call() == E.MLA_ERR_CUDA, name
+        assert E.last_cuda_error() != 0, name
 
 
 C_USER = r"""

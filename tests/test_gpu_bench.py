@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_bench_prints_one_contract_line():
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "200", "--warmup", "3",
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "20", "--warmup", "3",
                         "--no-sweep", "--no-cpu-baseline"], capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
@@ -23,13 +23,23 @@ def test_bench_prints_one_contract_line():
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
               "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
         assert k in d, k
-    assert d["n_gpus"] == 1 and d["steps"] == 200 and d["warmup"] == 3 and d["higher_is_better"] is False
-    assert 0.5 < d["value"] < 100.0
-    assert d["config"]["workload"] == "split_boundary_t64_h16_rope"
+    assert d["n_gpus"] == 1 and d["steps"] == 20 and d["warmup"] == 3 and d["higher_is_better"] is False
+    assert d["config"]["workload"] == "batch_t8192_h16_pdl_fp8"
+    # the reference arm prints the same config apart from its implementation
+    ref = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "3"], capture_output=True, text=True, timeout=900)
+    assert ref.returncode == 0, ref.stderr[-2000:]
+    rc = json.loads(ref.stdout.strip().splitlines()[-1])["config"]
+    assert {k: v for k, v in rc.items() if k != "implementation"} == \
+        {k: v for k, v in d["config"].items() if k != "implementation"}
+    assert 10.0 < d["value"] < 500.0
     rf = d["roofline"]
     assert rf["bound"] == "hbm" and rf["unit"] == "GB/s" and 0 < rf["frac"] < 1.5
     assert abs(rf["achieved"] / rf["peak"] - rf["frac"]) < 1e-3
+    assert len(d["timing"]["region_us_per_call_sorted"]) == d["timing"]["regions"] >= 10
     e = d["e2e"]
     assert e["value"] > d["value"] and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
-    assert d["gpu_launches"] == 200
-    assert d["launch_floor_us"] > 0 and d["l2_warm"]["us_per_call"] > 0
+    assert d["gpu_launches"] == 20
+    assert d["launch_floor_us"] > 0
+    bp = d["behind_producer"]
+    assert bp["producer_us"] > 0 and bp["epilogue_increment_pdl_us"] > 0

@@ -17,7 +17,7 @@ from parity_util import assert_same, check_workload, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
-FORCE = [0, E.MLA_FLAG_FORCE_SPLIT, E.MLA_FLAG_FORCE_ROWS]
+FORCE = [0, E.MLA_FLAG_FORCE_SPLIT, E.MLA_FLAG_FORCE_ROWS, E.MLA_FLAG_FORCE_TOKEN]
 
 
 # ---- the named workloads at their full sizes, in the launch configuration the bench times
@@ -33,7 +33,7 @@ def test_large_batch_behind_producer_with_pdl_matches_oracle():
     check_workload(w, producer=True)
 
 
-# ---- both kernels on the same inputs: bitwise identical (row split vs one warp per row)
+# ---- every kernel on the same inputs: bitwise identical (row split, single token, large batch)
 
 @pytest.mark.parametrize("T", [1, 7, 64, 65, 300])
 @pytest.mark.parametrize("flags", [0, W.FLAG_ROPE, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8,
@@ -59,6 +59,43 @@ def test_flag_combinations_and_shapes(flags, T, H):
                q_nope_row=520, q_pe_row=65, kv_c_row=1024, kv_c_offset=504, k_pe_row=67)
     for f in FORCE:
         check_workload(w, extra_flags=f)
+
+
+# ---- the single-token path (PR #53526 in the PR #54896 report's 关联脉络)
+
+@pytest.mark.parametrize("flags", list(range(8)))
+@pytest.mark.parametrize("H", [1, 16, 27, 28, 128])
+def test_single_token_behind_producer(flags, H):
+    """T = 1 through the plan's own choice (one block for H + 1 <= 28 rows),
+    launched with PDL behind the synthetic producer, every flag combination."""
+    assert E.mla_epilogue_plan(1, H, flags).mode == E.MLA_MODE_TOKEN
+    w = W.make("token", 1, H, flags, seed=600 + H * 8 + flags, num_blocks=2, std=2.0, rope_rows=1024,
+               scale=0.05, cache_fill="random")
+    check_workload(w, producer=True)
+    check_workload(w)
+
+
+# ---- inputs off the 16-byte grid take the scalar pe / table paths
+
+def _shift_view(t: torch.Tensor, elems: int) -> torch.Tensor:
+    """The same values in a buffer whose first element sits `elems` elements
+    past a 16-byte boundary (contiguous rows, same strides)."""
+    flat = torch.empty(t.numel() + elems, dtype=t.dtype)
+    out = flat[elems:].view(t.shape)
+    out.copy_(t)
+    return out
+
+
+@pytest.mark.parametrize("force", FORCE)
+@pytest.mark.parametrize("T", [1, 9, 300])
+def test_unaligned_pe_rows_and_table(force, T):
+    w = W.make("unaligned", T, 16, W.FLAG_ROPE | W.FLAG_Q_FP8, seed=70 + T, num_blocks=8, std=2.0, rope_rows=512,
+               scale=0.05, cache_fill="random")
+    w.q_pe = _shift_view(w.q_pe.contiguous(), 1)     # 2-byte aligned rows
+    w.k_pe = _shift_view(w.k_pe.contiguous(), 3)
+    w.cos_sin = _shift_view(w.cos_sin, 1)            # 4-byte aligned table rows
+    assert w.q_pe.data_ptr() % 16 and w.k_pe.data_ptr() % 16 and w.cos_sin.data_ptr() % 16
+    check_workload(w, extra_flags=force)
 
 
 def test_prefill_strided_views_are_really_strided():
