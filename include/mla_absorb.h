@@ -36,11 +36,6 @@
 extern "C" {
 #endif
 
-/* bit the kernel ORs into *status when one of its bounded waits on a copy or
- * on the tensor cores ran out: the outputs are then incomplete.  No such wait
- * is expected ever to run out. */
-#define MLA_STATUS_TIMEOUT 4
-
 /*
  * mla_absorb_launch
  *   q_nope_c  bf16 [T, H, 128] at element strides (stride_t, stride_h, 1): the

@@ -70,6 +70,9 @@ typedef enum mla_status {
 /* bits the kernel ORs into *status */
 #define MLA_STATUS_SLOT_RANGE 1  /* some slot_mapping[t] >= num_blocks*block_size: that cache row was not written */
 #define MLA_STATUS_POS_RANGE  2  /* some positions[t] outside [0, rope_rows): that token's rows were not rotated */
+#define MLA_STATUS_TIMEOUT    4  /* a bounded wait inside a kernel (on a copy, a barrier or the tensor cores)
+                                    ran out: the outputs are incomplete.  No such wait is expected ever to run
+                                    out; the kernel returns instead of hanging */
 
 /* Kernel choice (mla_plan.mode). */
 #define MLA_MODE_SPLIT 1 /* small T: 68 threads per 576-wide row, 64 with one 16-byte nope chunk each and 4 with

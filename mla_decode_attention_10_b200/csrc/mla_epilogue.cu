@@ -432,8 +432,9 @@ mla_status mla_epilogue_launch(
     return MLA_ERR_ALIGNMENT;
 
   // ---- plan and launch
+  int dev = 0;
   int32_t sms = 0;
-  mla_status s = mla::current_device(nullptr, &sms);
+  mla_status s = mla::current_device(&dev, &sms);
   if (s != MLA_OK) return s;
   mla_plan plan;
   s = make_plan(T, H, flags, sms, &plan);
@@ -477,7 +478,7 @@ mla_status mla_epilogue_launch(
   } else if (plan.mode == MLA_MODE_TOKEN) {
     fn = mla::kTokenKernels[k];
   } else {
-    s = mla::rows_kernel(k, &fn, &smem);
+    s = mla::rows_kernel(k, dev, &fn, &smem);
     if (s != MLA_OK) return s;
   }
 

@@ -11,8 +11,8 @@ namespace mla {
 
 // Upper limits (and defaults) of the tuning knobs mla_epilogue_set_tuning
 // clamps to.
-constexpr int kRowsMaxBlocksPerSm = 6;
-constexpr int kRowsMaxConsumerWarps = 8;
+constexpr int kRowsMaxBlocksPerSm = 1;     // persistent: one block per SM (184 KB of shared memory)
+constexpr int kRowsMaxConsumerWarps = 16;  // consumer warps beside the producer warp
 constexpr int kRowsDefaultWarps = 8;
 
 // Grid and block of a ROWS launch over `rows` rows.
@@ -20,7 +20,7 @@ void rows_plan(int64_t rows, bool qf8, bool kvf8, int32_t sm_count, int32_t bloc
                mla_plan* p);
 
 // The ROWS kernel for flags & 7 and its dynamic shared memory; makes the
-// kernel's shared-memory opt-in on the current device the first time.
-mla_status rows_kernel(int flag_bits, const void** fn, size_t* smem_bytes);
+// kernel's shared-memory opt-in on device `dev` the first time.
+mla_status rows_kernel(int flag_bits, int dev, const void** fn, size_t* smem_bytes);
 
 }  // namespace mla

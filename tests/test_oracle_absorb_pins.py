@@ -144,3 +144,31 @@ def test_zero_tokens_and_bad_flags():
     w = W.make_absorb("f", 2, 2, 0, seed=1)
     with pytest.raises(ValueError):
         oracle.absorb_run(w.q_nope_c, w.w_uk, w.q_pe, W.FLAG_KV_FP8)
+
+
+@pytest.mark.parametrize("flags", [W.FLAG_ROPE, W.FLAG_ROPE | W.FLAG_Q_FP8])
+def test_positions_out_of_range_leave_pe_unrotated(flags):
+    """The slot/position rule of the epilogue, on the absorbed rows: a
+    position outside [0, rope_rows) sets status bit 2 and leaves that token's
+    pe half unrotated (the bf16 input bits, or the e4m3 bytes of x / scale);
+    tokens in range are rotated.  The table is a quarter turn everywhere
+    (cos 0, sin 1), so a rotated pair (a, b) is exactly (-b, a) and the
+    expected values need no rounding of a product."""
+    T, H, rows = 6, 3, 8
+    w = W.make_absorb("posrule", T, H, flags, seed=21, rope_rows=rows, scale=0.25)
+    w.cos_sin = torch.cat((torch.zeros(rows, 32), torch.ones(rows, 32)), 1).contiguous()
+    w.positions = torch.tensor([0, -1, rows, 3, 2 ** 31 - 1, rows - 1], dtype=torch.int32)
+    q, st = _run(w)
+    assert st == oracle.STATUS_POS_RANGE
+    a, b = w.q_pe[..., :32], w.q_pe[..., 32:]
+    rotated = torch.cat((-b, a), -1)
+    for t in range(T):
+        inside = 0 <= int(w.positions[t]) < rows
+        want = rotated[t] if inside else w.q_pe[t]
+        if flags & W.FLAG_Q_FP8:
+            # x / 0.25 is exact (a power of two), so torch's cast of the
+            # quotient is the e4m3 byte of the definition
+            ref = (want.float() / 0.25).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+            assert torch.equal(q[t, :, 512:], ref), t
+        else:
+            assert torch.equal(_bits(q[t, :, 512:]), _bits(want)), t
