@@ -486,13 +486,15 @@ def decode_floors(hx, device, peak, calls=200, reps=7):
 
 
 def launch_to_end(hx, device, names=("decode_sweep_t1_h16_rope_fp8", "decode_sweep_t4_h16_rope_fp8",
-                                     "decode_sweep_t64_h16_rope_fp8"), iters=1000):
+                                     "decode_sweep_t64_h16_rope_fp8"), iters=1000, sleep_cycles=400_000):
     """Device time from an event recorded just before one isolated launch to
     one recorded just after it, for the epilogue and for the empty kernel of
-    the same grid: median (and 10th / 90th percentile) of `iters` launches,
-    each preceded, outside its event pair, by a write of twice the L2 (which
-    also keeps the launch queued ahead of the GPU, so the pair holds the
-    device-side launch, the kernel and its completion, not host overhead)."""
+    the same grid: median (and 10th / 90th percentile) of `iters` launches.
+    Before each event pair, outside it, the stream writes twice the L2 (cold
+    inputs) and then sleeps on the GPU for about 200 us, so the host has
+    queued the launch and the closing event before the opening event
+    executes: the pair holds the device-side launch, the kernel and its
+    completion, not host overhead."""
     E, stream = hx.E, hx.stream
     buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=device)
     out = []
@@ -508,6 +510,7 @@ def launch_to_end(hx, device, names=("decode_sweep_t1_h16_rope_fp8", "decode_swe
                 with torch.cuda.stream(stream):
                     for i in range(base, min(iters, base + 100)):
                         buf.fill_(i)
+                        torch.cuda._sleep(sleep_cycles)
                         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                         e0.record(stream)
                         fn(i)

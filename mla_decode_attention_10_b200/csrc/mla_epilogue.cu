@@ -157,53 +157,92 @@ __device__ __forceinline__ void store_pe8(uint8_t* row, int j, const uint4 lo, c
 // small-batch kernels (SPLIT: NC = 1, TOKEN: NC = 2 nope chunks per thread)
 // ------------------------------------------------------------------------------------
 
-template <int NC, bool FP8, bool ROPE, bool FAST>
-__device__ __forceinline__ void small_cache_row(const Args& a, int64_t t, bool pe, int part, const Divisor& d) {
+// A row's e4m3 scale: its load is issued with the row's other loads and the
+// divisor is made only when the stores need it, so the scale adds no step
+// to the row's chain of dependent loads.
+template <bool FP8>
+__device__ __forceinline__ float scale_of(const float* scale) {
+  if constexpr (FP8) return __ldg(scale);
+  return 1.0f;
+}
+
+template <bool FP8>
+__device__ __forceinline__ Divisor divisor_from(float scale) {
+  Divisor d{};
+  d.fast = true;
+  if constexpr (FP8) d = make_divisor(scale);
+  return d;
+}
+
+// Stores of one thread's share of a row, the quotient path chosen from the
+// scale: the corrected reciprocal unless the scale is outside [2^-64, 2^64].
+template <int NC, bool FP8, bool ROPE>
+__device__ __forceinline__ void store_part(uint8_t* dst, bool pe, int part, const uint4 (&v)[NC], const uint4& lo,
+                                           const uint4& hi, const Rot8& rot, float scale) {
   constexpr int kNopeLanes = 64 / NC;
-  const int64_t slot = __ldg(a.slots + t);
-  const bool in_range = slot >= 0 && slot < a.cache_rows;
-  uint8_t* dst = a.cache + (in_range ? slot : 0) * (FP8 ? kRow : 2 * kRow);
-  if (!pe) {
-    const uint16_t* src = a.kv_c + t * a.kv_st;
-    uint4 v[NC];
+  const Divisor d = divisor_from<FP8>(scale);
+  if (!FP8 || d.fast) {
+    if (!pe) {
 #pragma unroll
-    for (int k = 0; k < NC; ++k) v[k] = ld_cg16(src + 8 * (part + k * kNopeLanes));
-    if (part == 0 && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
-    if (in_range) {
-#pragma unroll
-      for (int k = 0; k < NC; ++k) store_nope<FP8, FAST>(dst, part + k * kNopeLanes, v[k], d);
+      for (int k = 0; k < NC; ++k) store_nope<FP8, true>(dst, part + k * kNopeLanes, v[k], d);
+    } else {
+      store_pe8<FP8, ROPE, true>(dst, part, lo, hi, rot, d);
     }
   } else {
-    const Rot8 rot = load_rot8<ROPE>(a, t, part);
-    if (ROPE && part == 0 && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
-    uint4 lo, hi;
-    load_pe8(a.k_pe + t * a.kp_st, part, a.kpe_vec != 0, lo, hi);
-    if (in_range) store_pe8<FP8, ROPE, FAST>(dst, part, lo, hi, rot, d);
+    if (!pe) {
+#pragma unroll
+      for (int k = 0; k < NC; ++k) store_nope<FP8, false>(dst, part + k * kNopeLanes, v[k], d);
+    } else {
+      store_pe8<FP8, ROPE, false>(dst, part, lo, hi, rot, d);
+    }
   }
 }
 
-template <int NC, bool FP8, bool ROPE, bool FAST>
-__device__ __forceinline__ void small_query_row(const Args& a, int64_t q, bool pe, int part, const Divisor& d) {
+template <int NC, bool FP8, bool ROPE>
+__device__ __forceinline__ void small_cache_row(const Args& a, int64_t t, bool pe, int part) {
   constexpr int kNopeLanes = 64 / NC;
+  const float scale = scale_of<FP8>(a.kv_scale);
+  const int64_t slot = __ldg(a.slots + t);
+  uint4 v[NC], lo = make_uint4(0, 0, 0, 0), hi = lo;
+  Rot8 rot;
+  rot.on = false;
+  if (!pe) {
+    const uint16_t* src = a.kv_c + t * a.kv_st;
+#pragma unroll
+    for (int k = 0; k < NC; ++k) v[k] = ld_cg16(src + 8 * (part + k * kNopeLanes));
+  } else {
+    rot = load_rot8<ROPE>(a, t, part);
+    load_pe8(a.k_pe + t * a.kp_st, part, a.kpe_vec != 0, lo, hi);
+  }
+  const bool in_range = slot >= 0 && slot < a.cache_rows;
+  if (part == 0) {
+    if (!pe && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
+    if (ROPE && pe && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
+  }
+  if (in_range) store_part<NC, FP8, ROPE>(a.cache + slot * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
+}
+
+template <int NC, bool FP8, bool ROPE>
+__device__ __forceinline__ void small_query_row(const Args& a, int64_t q, bool pe, int part) {
+  constexpr int kNopeLanes = 64 / NC;
+  const float scale = scale_of<FP8>(a.q_scale);
   const int64_t t = div_heads(a, q);
   const int64_t h = q - t * a.H;
-  uint8_t* dst = a.q_out + q * (FP8 ? kRow : 2 * kRow);
+  uint4 v[NC], lo = make_uint4(0, 0, 0, 0), hi = lo;
+  Rot8 rot;
+  rot.on = false;
   if (!pe) {
     const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh;
     pdl_wait();
-    uint4 v[NC];
 #pragma unroll
     for (int k = 0; k < NC; ++k) v[k] = ld_cg16(src + 8 * (part + k * kNopeLanes));
-#pragma unroll
-    for (int k = 0; k < NC; ++k) store_nope<FP8, FAST>(dst, part + k * kNopeLanes, v[k], d);
   } else {
     const uint16_t* src = a.q_pe + t * a.qp_st + h * a.qp_sh;
-    const Rot8 rot = load_rot8<ROPE>(a, t, part);
+    rot = load_rot8<ROPE>(a, t, part);
     pdl_wait();
-    uint4 lo, hi;
     load_pe8(src, part, a.qpe_vec != 0, lo, hi);
-    store_pe8<FP8, ROPE, FAST>(dst, part, lo, hi, rot, d);
   }
+  store_part<NC, FP8, ROPE>(a.q_out + q * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
 }
 
 template <int NC, bool QF8, bool KVF8, bool ROPE>
@@ -218,22 +257,10 @@ __global__ void __launch_bounds__(kSmallMaxThreads) mla_epilogue_small_kernel(co
   const int part = pe ? (u & 3) : (u % kNopeLanes);
   const int64_t g = static_cast<int64_t>(blockIdx.x) * R + r;
   if (g < a.rows) {
-    // the divisor of the row's scale (read before any wait); quotients take
-    // the corrected-reciprocal path unless the scale is outside [2^-64, 2^64]
     if (g < a.T) {
-      const Divisor d = divisor_of<KVF8>(a.kv_scale);
-      if (d.fast) {
-        small_cache_row<NC, KVF8, ROPE, true>(a, g, pe, part, d);
-      } else {
-        small_cache_row<NC, KVF8, ROPE, false>(a, g, pe, part, d);
-      }
+      small_cache_row<NC, KVF8, ROPE>(a, g, pe, part);
     } else {
-      const Divisor d = divisor_of<QF8>(a.q_scale);
-      if (d.fast) {
-        small_query_row<NC, QF8, ROPE, true>(a, g - a.T, pe, part, d);
-      } else {
-        small_query_row<NC, QF8, ROPE, false>(a, g - a.T, pe, part, d);
-      }
+      small_query_row<NC, QF8, ROPE>(a, g - a.T, pe, part);
     }
   }
   pdl_trigger();
@@ -366,7 +393,7 @@ void mla_epilogue_set_tuning(const mla_tuning* t) {
         t->split_rows_per_block < mla::kSmallMaxRowsPerBlock ? t->split_rows_per_block : mla::kSmallMaxRowsPerBlock;
   if (t->rows_warps_per_block > 0)
     g_tuning.rows_warps_per_block =
-        t->rows_warps_per_block < mla::kRowsMaxConsumerWarps ? t->rows_warps_per_block : mla::kRowsMaxConsumerWarps;
+        t->rows_warps_per_block < mla::kRowsMaxWarps ? t->rows_warps_per_block : mla::kRowsMaxWarps;
   if (t->rows_blocks_per_sm > 0)
     g_tuning.rows_blocks_per_sm =
         t->rows_blocks_per_sm < mla::kRowsMaxBlocksPerSm ? t->rows_blocks_per_sm : mla::kRowsMaxBlocksPerSm;
@@ -432,9 +459,8 @@ mla_status mla_epilogue_launch(
     return MLA_ERR_ALIGNMENT;
 
   // ---- plan and launch
-  int dev = 0;
   int32_t sms = 0;
-  mla_status s = mla::current_device(&dev, &sms);
+  mla_status s = mla::current_device(nullptr, &sms);
   if (s != MLA_OK) return s;
   mla_plan plan;
   s = make_plan(T, H, flags, sms, &plan);
@@ -478,7 +504,7 @@ mla_status mla_epilogue_launch(
   } else if (plan.mode == MLA_MODE_TOKEN) {
     fn = mla::kTokenKernels[k];
   } else {
-    s = mla::rows_kernel(k, dev, &fn, &smem);
+    s = mla::rows_kernel(k, plan.threads_per_block / 32, &fn, &smem);
     if (s != MLA_OK) return s;
   }
 

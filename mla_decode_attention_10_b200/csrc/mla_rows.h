@@ -11,16 +11,16 @@ namespace mla {
 
 // Upper limits (and defaults) of the tuning knobs mla_epilogue_set_tuning
 // clamps to.
-constexpr int kRowsMaxBlocksPerSm = 1;     // persistent: one block per SM (184 KB of shared memory)
-constexpr int kRowsMaxConsumerWarps = 16;  // consumer warps beside the producer warp
+constexpr int kRowsMaxBlocksPerSm = 5;  // resident blocks per SM the kernel is compiled for
+constexpr int kRowsMaxWarps = 8;        // warps per block (each with its own 4.5 KB row ring)
 constexpr int kRowsDefaultWarps = 8;
 
 // Grid and block of a ROWS launch over `rows` rows.
 void rows_plan(int64_t rows, bool qf8, bool kvf8, int32_t sm_count, int32_t blocks_per_sm, int32_t warps_per_block,
                mla_plan* p);
 
-// The ROWS kernel for flags & 7 and its dynamic shared memory; makes the
-// kernel's shared-memory opt-in on device `dev` the first time.
-mla_status rows_kernel(int flag_bits, int dev, const void** fn, size_t* smem_bytes);
+// The ROWS kernel for flags & 7 and its dynamic shared memory for blocks of
+// `warps` warps.
+mla_status rows_kernel(int flag_bits, int warps, const void** fn, size_t* smem_bytes);
 
 }  // namespace mla

@@ -100,14 +100,14 @@ def test_unaligned_pe_rows_and_table(force, T):
 
 # ---- the large-batch kernel's block shape: any number of consumer warps
 
-@pytest.mark.parametrize("warps", [1, 3, 8, 16])
-def test_rows_kernel_consumer_warp_counts(warps):
-    """Tiles of 32 rows shared by 1 .. 16 consumer warps (a warp takes rows
-    w, w + W, ...), many tiles per block so the four-stage ring wraps."""
+@pytest.mark.parametrize("warps", [1, 3, 8])
+def test_rows_kernel_warp_counts(warps):
+    """Blocks of 1 .. 8 warps; every warp walks many rows, so its four-slot
+    ring wraps many times."""
     old = E.mla_epilogue_get_tuning()
     try:
         E.mla_epilogue_set_tuning(rows_warps_per_block=warps)
-        assert E.mla_epilogue_plan(777, 12, E.MLA_FLAG_FORCE_ROWS).threads_per_block == 32 * (1 + warps)
+        assert E.mla_epilogue_plan(777, 12, E.MLA_FLAG_FORCE_ROWS).threads_per_block == 32 * warps
         w = W.make("warps", 777, 12, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8, seed=90 + warps, num_blocks=64,
                    std=2.0, rope_rows=2048, scale=0.05, cache_fill="random")
         check_workload(w, extra_flags=E.MLA_FLAG_FORCE_ROWS)
