@@ -64,8 +64,7 @@ typedef enum mla_status {
 #define MLA_FLAG_KV_FP8      4u  /* cache is e4m3 bytes, scaled by *kv_scale (needs kv_scale) */
 #define MLA_FLAG_PDL         8u  /* launch as a programmatic dependent of the previous kernel on `stream` */
 #define MLA_FLAG_FORCE_SPLIT 16u /* use MLA_MODE_SPLIT whatever T is (tests, tuning) */
-#define MLA_FLAG_FORCE_ROWS  32u /* use MLA_MODE_ROWS whatever T is (tests, tuning) */
-#define MLA_FLAG_FORCE_TOKEN 64u /* use MLA_MODE_TOKEN whatever T is (tests, tuning); at most one FORCE flag */
+#define MLA_FLAG_FORCE_ROWS  32u /* use MLA_MODE_ROWS whatever T is (tests, tuning); not with FORCE_SPLIT */
 
 /* bits the kernel ORs into *status */
 #define MLA_STATUS_SLOT_RANGE 1  /* some slot_mapping[t] >= num_blocks*block_size: that cache row was not written */
@@ -76,10 +75,10 @@ typedef enum mla_status {
 
 /* Kernel choice (mla_plan.mode). */
 #define MLA_MODE_SPLIT 1 /* small T: 68 threads per 576-wide row, 64 with one 16-byte nope chunk each and 4 with
-                            eight RoPE pairs each (16-byte loads); rows_per_block rows per block */
-#define MLA_MODE_ROWS  2 /* large T: persistent blocks, grid a multiple of the SM count */
-#define MLA_MODE_TOKEN 3 /* T == 1: 36 threads per row (two nope chunks each), every row of the token in one
-                            block when H + 1 <= 28 */
+                            eight RoPE pairs each (16-byte loads); threads map to rows by their index in the grid
+                            and blocks are sized to about one per SM (one-warp blocks for a single token) */
+#define MLA_MODE_ROWS  2 /* large T: one warp per row, grid-stride, slot and position loaded one row ahead;
+                            grid sized to the resident blocks */
 
 /*
  * mla_epilogue_launch -- the whole epilogue in one kernel launch.
@@ -156,13 +155,14 @@ MLA_API mla_status mla_epilogue_launch(
  * the current device, without launching anything.  Host only; needs the
  * device's SM count, which it reads once per device (sm_count <= 0 lets the
  * caller pass it instead: `sm_count` > 0 is used as given and no CUDA call is
- * made).  Returns MLA_ERR_INVALID_ARG for T < 1, H < 1 or more than one FORCE flag.
+ * made).  Returns MLA_ERR_INVALID_ARG for T < 1, H < 1 or both FORCE flags.
  */
 typedef struct mla_plan {
   int32_t mode;              /* MLA_MODE_SPLIT or MLA_MODE_ROWS */
   int32_t threads_per_block;
   int64_t blocks;
-  int32_t rows_per_block;    /* SPLIT, TOKEN: rows one block covers; ROWS: 1 */
+  int32_t rows_per_block;    /* ROWS: 1 (one row per warp at a time); SPLIT: 0 (rows spread over blocks by
+                                thread index, 68 threads a row) */
   int32_t sm_count;
 } mla_plan;
 
@@ -175,19 +175,20 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  * sizes or hardware (PR #54896 report, 风险与影响 "risks" item 2).  On B200
  * the split kernel stays faster than the rows kernel up to about 4.6 K rows
  * (T * (H + 1)) whatever H is (measured for H = 8, 16, 32, 128), so the
- * default threshold counts rows, not tokens.  A value <= 0 keeps the current
- * setting.
+ * default threshold counts rows, not tokens.
  *   split_max_rows       T * (H + 1) at or below which MLA_MODE_SPLIT is used (default 4608)
- *   split_rows_per_block rows per block in MLA_MODE_SPLIT (block = 68 * this), at most 15
- *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8
+ *   split_threads_per_block threads per block in MLA_MODE_SPLIT, rounded up to a multiple of
+ *                        32, at most 1024; 0 (default) sizes blocks to about one per SM;
+ *                        a negative value restores the default
+ *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8 (default 8)
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
- *                        the number the kernel's register cap keeps resident
- *                        (6 with an e4m3 output, 5 without)
- * Larger values are clamped to those limits.
+ *                        5, the number the kernel's register cap keeps resident
+ *                        (default 5)
+ * Larger values are clamped to those limits; 0 keeps the current setting.
  */
 typedef struct mla_tuning {
   int64_t split_max_rows;
-  int32_t split_rows_per_block;
+  int32_t split_threads_per_block;
   int32_t rows_warps_per_block;
   int32_t rows_blocks_per_sm;
 } mla_tuning;

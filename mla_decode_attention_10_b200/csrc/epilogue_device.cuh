@@ -44,7 +44,6 @@ struct Args {
   uint8_t* q_out;
   uint8_t* cache;
   int32_t* status;
-  int32_t rows_per_block;  // small-batch kernels: rows one block covers
   // 16-byte vector access is possible (base 16-byte aligned, strides
   // multiples of 8 elements): q_pe rows, k_pe rows, cos_sin rows
   int32_t qpe_vec, kpe_vec, tab_vec;

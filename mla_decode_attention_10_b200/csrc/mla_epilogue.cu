@@ -14,16 +14,19 @@
 //     nope chunk each (8 values); 4 of them each own the pe octets 8j..8j+7
 //     and 32+8j..32+8j+7, so one thread holds both members of its 8 RoPE
 //     pairs (i, i+32) and rotates them without shuffles, with 16-byte loads
-//     and 16-byte (bf16) or 8-byte (e4m3) stores.  A block holds R rows:
-//     first the 64R nope threads, then the 4R pe threads, so every warp has
-//     one role.
-//   TOKEN (T == 1): the same row code with 32 nope threads per row, two
-//     chunks each (c and c + 32), so all H + 1 rows of the token fit in one
-//     block for H <= 27: one block, one position, one table row, a single
-//     wave of loads (the num_tokens == 1 case of PR #53526, 关联脉络).
+//     and 16-byte (bf16) or 8-byte (e4m3) stores.  Threads map to work by
+//     their index in the grid: the first 64 * rows threads are the nope
+//     threads of all rows, the next 4 * rows the pe threads (eight rows per
+//     warp), so every warp has one role and the block size is free.  At
+//     decode sizes the latency is lowest when the work is spread over as
+//     many SMs as there are (measured on B200: one 17-row token in 37
+//     one-warp blocks is about 0.9 us faster than in one to three blocks),
+//     so the plan sizes blocks to give about one block per SM; for T = 1
+//     that is one-warp blocks (the num_tokens == 1 case of PR #53526,
+//     关联脉络).
 //   ROWS (large T): mla_rows.cu.
 //
-// In SPLIT and TOKEN every thread computes its addresses and loads its slot,
+// In SPLIT every thread computes its addresses and loads its slot,
 // position, table entries and scale before griddepcontrol.wait; after the
 // wait a query-row thread has one load -> convert -> store left (PR #54896
 // report, 实现拆解 item 2).  Cache rows never wait.  Every thread issues
@@ -43,9 +46,7 @@
 namespace mla {
 
 constexpr int kSmallMaxThreads = 1024;
-constexpr int kSmallMaxRowsPerBlock = 15;  // 68 * 15 = 1020 threads
-constexpr int kTokenLanesPerRow = 36;      // 32 nope threads (two chunks each) + 4 pe threads
-constexpr int kTokenMaxRowsPerBlock = kSmallMaxThreads / kTokenLanesPerRow;  // 28
+constexpr int kSmallThreadsPerRow = 68;  // 64 nope threads + 4 pe threads
 
 // Nope chunk `chunk` (8 values) of a row: 16 bytes in, 16 (bf16) or 8 (e4m3) out.
 template <bool FP8, bool FAST>
@@ -154,7 +155,7 @@ __device__ __forceinline__ void store_pe8(uint8_t* row, int j, const uint4 lo, c
 }
 
 // ------------------------------------------------------------------------------------
-// small-batch kernels (SPLIT: NC = 1, TOKEN: NC = 2 nope chunks per thread)
+// small-batch kernel
 // ------------------------------------------------------------------------------------
 
 // A row's e4m3 scale: its load is issued with the row's other loads and the
@@ -176,40 +177,34 @@ __device__ __forceinline__ Divisor divisor_from(float scale) {
 
 // Stores of one thread's share of a row, the quotient path chosen from the
 // scale: the corrected reciprocal unless the scale is outside [2^-64, 2^64].
-template <int NC, bool FP8, bool ROPE>
-__device__ __forceinline__ void store_part(uint8_t* dst, bool pe, int part, const uint4 (&v)[NC], const uint4& lo,
+template <bool FP8, bool ROPE>
+__device__ __forceinline__ void store_part(uint8_t* dst, bool pe, int part, const uint4& v, const uint4& lo,
                                            const uint4& hi, const Rot8& rot, float scale) {
-  constexpr int kNopeLanes = 64 / NC;
   const Divisor d = divisor_from<FP8>(scale);
   if (!FP8 || d.fast) {
     if (!pe) {
-#pragma unroll
-      for (int k = 0; k < NC; ++k) store_nope<FP8, true>(dst, part + k * kNopeLanes, v[k], d);
+      store_nope<FP8, true>(dst, part, v, d);
     } else {
       store_pe8<FP8, ROPE, true>(dst, part, lo, hi, rot, d);
     }
   } else {
     if (!pe) {
-#pragma unroll
-      for (int k = 0; k < NC; ++k) store_nope<FP8, false>(dst, part + k * kNopeLanes, v[k], d);
+      store_nope<FP8, false>(dst, part, v, d);
     } else {
       store_pe8<FP8, ROPE, false>(dst, part, lo, hi, rot, d);
     }
   }
 }
 
-template <int NC, bool FP8, bool ROPE>
+template <bool FP8, bool ROPE>
 __device__ __forceinline__ void small_cache_row(const Args& a, int64_t t, bool pe, int part) {
-  constexpr int kNopeLanes = 64 / NC;
   const float scale = scale_of<FP8>(a.kv_scale);
   const int64_t slot = __ldg(a.slots + t);
-  uint4 v[NC], lo = make_uint4(0, 0, 0, 0), hi = lo;
+  uint4 v = make_uint4(0, 0, 0, 0), lo = v, hi = v;
   Rot8 rot;
   rot.on = false;
   if (!pe) {
-    const uint16_t* src = a.kv_c + t * a.kv_st;
-#pragma unroll
-    for (int k = 0; k < NC; ++k) v[k] = ld_cg16(src + 8 * (part + k * kNopeLanes));
+    v = ld_cg16(a.kv_c + t * a.kv_st + 8 * part);
   } else {
     rot = load_rot8<ROPE>(a, t, part);
     load_pe8(a.k_pe + t * a.kp_st, part, a.kpe_vec != 0, lo, hi);
@@ -219,66 +214,60 @@ __device__ __forceinline__ void small_cache_row(const Args& a, int64_t t, bool p
     if (!pe && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
     if (ROPE && pe && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
   }
-  if (in_range) store_part<NC, FP8, ROPE>(a.cache + slot * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
+  if (in_range) store_part<FP8, ROPE>(a.cache + slot * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
 }
 
-template <int NC, bool FP8, bool ROPE>
+template <bool FP8, bool ROPE>
 __device__ __forceinline__ void small_query_row(const Args& a, int64_t q, bool pe, int part) {
-  constexpr int kNopeLanes = 64 / NC;
   const float scale = scale_of<FP8>(a.q_scale);
   const int64_t t = div_heads(a, q);
   const int64_t h = q - t * a.H;
-  uint4 v[NC], lo = make_uint4(0, 0, 0, 0), hi = lo;
+  uint4 v = make_uint4(0, 0, 0, 0), lo = v, hi = v;
   Rot8 rot;
   rot.on = false;
   if (!pe) {
-    const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh;
+    const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh + 8 * part;
     pdl_wait();
-#pragma unroll
-    for (int k = 0; k < NC; ++k) v[k] = ld_cg16(src + 8 * (part + k * kNopeLanes));
+    v = ld_cg16(src);
   } else {
     const uint16_t* src = a.q_pe + t * a.qp_st + h * a.qp_sh;
     rot = load_rot8<ROPE>(a, t, part);
     pdl_wait();
     load_pe8(src, part, a.qpe_vec != 0, lo, hi);
   }
-  store_part<NC, FP8, ROPE>(a.q_out + q * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
+  store_part<FP8, ROPE>(a.q_out + q * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
 }
 
-template <int NC, bool QF8, bool KVF8, bool ROPE>
+template <bool QF8, bool KVF8, bool ROPE>
 __global__ void __launch_bounds__(kSmallMaxThreads) mla_epilogue_small_kernel(const Args a) {
-  constexpr int kNopeLanes = 64 / NC;
-  const int R = a.rows_per_block;
-  const int tid = static_cast<int>(threadIdx.x);
-  const int nope_threads = kNopeLanes * R;
-  const bool pe = tid >= nope_threads;
-  const int u = pe ? tid - nope_threads : tid;
-  const int r = pe ? (u >> 2) : (u / kNopeLanes);
-  const int part = pe ? (u & 3) : (u % kNopeLanes);
-  const int64_t g = static_cast<int64_t>(blockIdx.x) * R + r;
+  // thread -> (row, part) by its index in the grid: nope threads of all rows
+  // first (64 per row), then pe threads (4 per row)
+  const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nope_threads = 64 * a.rows;
+  const bool pe = gt >= nope_threads;
+  const int64_t u = pe ? gt - nope_threads : gt;
+  const int64_t g = pe ? (u >> 2) : (u >> 6);
+  const int part = static_cast<int>(pe ? (u & 3) : (u & 63));
   if (g < a.rows) {
     if (g < a.T) {
-      small_cache_row<NC, KVF8, ROPE>(a, g, pe, part);
+      small_cache_row<KVF8, ROPE>(a, g, pe, part);
     } else {
-      small_query_row<NC, QF8, ROPE>(a, g - a.T, pe, part);
+      small_query_row<QF8, ROPE>(a, g - a.T, pe, part);
     }
   }
   pdl_trigger();
 }
 
 // kernel tables indexed by (ROPE, Q_FP8, KV_FP8) = flags & 7
-template <int NC, int F>
+template <int F>
 const void* small_kernel_for() {
-  return reinterpret_cast<const void*>(&mla_epilogue_small_kernel<NC, (F & MLA_FLAG_Q_FP8) != 0,
-                                                                  (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
+  return reinterpret_cast<const void*>(
+      &mla_epilogue_small_kernel<(F & MLA_FLAG_Q_FP8) != 0, (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
 }
 
-const void* const kSplitKernels[8] = {small_kernel_for<1, 0>(), small_kernel_for<1, 1>(), small_kernel_for<1, 2>(),
-                                      small_kernel_for<1, 3>(), small_kernel_for<1, 4>(), small_kernel_for<1, 5>(),
-                                      small_kernel_for<1, 6>(), small_kernel_for<1, 7>()};
-const void* const kTokenKernels[8] = {small_kernel_for<2, 0>(), small_kernel_for<2, 1>(), small_kernel_for<2, 2>(),
-                                      small_kernel_for<2, 3>(), small_kernel_for<2, 4>(), small_kernel_for<2, 5>(),
-                                      small_kernel_for<2, 6>(), small_kernel_for<2, 7>()};
+const void* const kSplitKernels[8] = {small_kernel_for<0>(), small_kernel_for<1>(), small_kernel_for<2>(),
+                                      small_kernel_for<3>(), small_kernel_for<4>(), small_kernel_for<5>(),
+                                      small_kernel_for<6>(), small_kernel_for<7>()};
 
 // ------------------------------------------------------------------------------------
 // host helpers shared by every launcher (mla_runtime.h)
@@ -322,45 +311,42 @@ mla_status current_device(int* dev_out, int32_t* sm_count) {
 namespace {
 
 constexpr uint32_t kKnownFlags = MLA_FLAG_ROPE | MLA_FLAG_Q_FP8 | MLA_FLAG_KV_FP8 | MLA_FLAG_PDL |
-                                 MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS | MLA_FLAG_FORCE_TOKEN;
-constexpr uint32_t kForceFlags = MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS | MLA_FLAG_FORCE_TOKEN;
+                                 MLA_FLAG_FORCE_SPLIT | MLA_FLAG_FORCE_ROWS;
 
-mla_tuning g_tuning = {4608, 8, mla::kRowsDefaultWarps, mla::kRowsMaxBlocksPerSm};
+mla_tuning g_tuning = {4608, 0, mla::kRowsDefaultWarps, mla::kRowsMaxBlocksPerSm};
 
 bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
 
 bool one_force_flag(uint32_t flags) {
-  const uint32_t f = flags & kForceFlags;
-  return (f & (f - 1)) == 0;
+  return !((flags & MLA_FLAG_FORCE_SPLIT) && (flags & MLA_FLAG_FORCE_ROWS));
+}
+
+// Threads per SPLIT block: the tuning value, or (0) the smallest multiple of
+// 32 that gives at most one block per SM, between 32 and 1024.
+int32_t split_threads(int64_t rows, int32_t sm_count) {
+  if (g_tuning.split_threads_per_block > 0) return g_tuning.split_threads_per_block;
+  const int64_t threads = mla::kSmallThreadsPerRow * rows;
+  int64_t per = (threads + sm_count - 1) / sm_count;
+  per = (per + 31) / 32 * 32;
+  return static_cast<int32_t>(per < 32 ? 32 : (per > mla::kSmallMaxThreads ? mla::kSmallMaxThreads : per));
 }
 
 mla_status make_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla_plan* p) {
   const int64_t rows = T * (H + 1);
-  int32_t mode;
-  if (flags & MLA_FLAG_FORCE_SPLIT) {
-    mode = MLA_MODE_SPLIT;
-  } else if (flags & MLA_FLAG_FORCE_ROWS) {
-    mode = MLA_MODE_ROWS;
-  } else if (flags & MLA_FLAG_FORCE_TOKEN) {
-    mode = MLA_MODE_TOKEN;
-  } else if (T == 1) {
-    mode = MLA_MODE_TOKEN;
-  } else {
-    mode = rows <= g_tuning.split_max_rows ? MLA_MODE_SPLIT : MLA_MODE_ROWS;
-  }
-  p->mode = mode;
+  const bool split = (flags & MLA_FLAG_FORCE_SPLIT)  ? true
+                     : (flags & MLA_FLAG_FORCE_ROWS) ? false
+                                                      : rows <= g_tuning.split_max_rows;
   p->sm_count = sm_count;
-  if (mode == MLA_MODE_SPLIT) {
-    const int32_t rpb = g_tuning.split_rows_per_block;
-    p->rows_per_block = rpb;
-    p->threads_per_block = (64 + 4) * rpb;
-    p->blocks = (rows + rpb - 1) / rpb;
-  } else if (mode == MLA_MODE_TOKEN) {
-    // all rows of one token in one block where they fit
-    const int64_t rpb = H + 1 < mla::kTokenMaxRowsPerBlock ? H + 1 : mla::kTokenMaxRowsPerBlock;
-    p->rows_per_block = static_cast<int32_t>(rpb);
-    p->threads_per_block = mla::kTokenLanesPerRow * static_cast<int32_t>(rpb);
-    p->blocks = (rows + rpb - 1) / rpb;
+  if (split) {
+    const int32_t tpb = split_threads(rows, sm_count);
+    p->mode = MLA_MODE_SPLIT;
+    p->rows_per_block = 0;
+    p->threads_per_block = tpb;
+    p->blocks = (mla::kSmallThreadsPerRow * rows + tpb - 1) / tpb;
+    if (p->blocks > INT_MAX) {  // a small tuned block size on a huge forced launch
+      p->threads_per_block = mla::kSmallMaxThreads;
+      p->blocks = (mla::kSmallThreadsPerRow * rows + mla::kSmallMaxThreads - 1) / mla::kSmallMaxThreads;
+    }
   } else {
     mla::rows_plan(rows, (flags & MLA_FLAG_Q_FP8) != 0, (flags & MLA_FLAG_KV_FP8) != 0, sm_count,
                    g_tuning.rows_blocks_per_sm, g_tuning.rows_warps_per_block, p);
@@ -388,9 +374,12 @@ int32_t mla_last_cuda_error(void) { return mla::g_last_cuda_error; }
 void mla_epilogue_set_tuning(const mla_tuning* t) {
   if (t == nullptr) return;
   if (t->split_max_rows > 0) g_tuning.split_max_rows = t->split_max_rows;
-  if (t->split_rows_per_block > 0)
-    g_tuning.split_rows_per_block =
-        t->split_rows_per_block < mla::kSmallMaxRowsPerBlock ? t->split_rows_per_block : mla::kSmallMaxRowsPerBlock;
+  if (t->split_threads_per_block > 0) {
+    const int32_t v = (t->split_threads_per_block + 31) / 32 * 32;
+    g_tuning.split_threads_per_block = v < mla::kSmallMaxThreads ? v : mla::kSmallMaxThreads;
+  } else if (t->split_threads_per_block < 0) {
+    g_tuning.split_threads_per_block = 0;  // back to the automatic block size
+  }
   if (t->rows_warps_per_block > 0)
     g_tuning.rows_warps_per_block =
         t->rows_warps_per_block < mla::kRowsMaxWarps ? t->rows_warps_per_block : mla::kRowsMaxWarps;
@@ -491,7 +480,6 @@ mla_status mla_epilogue_launch(
   a.q_out = static_cast<uint8_t*>(q_out);
   a.cache = static_cast<uint8_t*>(cache);
   a.status = status;
-  a.rows_per_block = plan.rows_per_block;
   a.qpe_vec = aligned(q_pe, 16) && (T == 1 || q_pe_stride_t % 8 == 0) && (H == 1 || q_pe_stride_h % 8 == 0);
   a.kpe_vec = aligned(k_pe, 16) && (T == 1 || k_pe_stride_t % 8 == 0);
   a.tab_vec = rope && aligned(cos_sin, 16);
@@ -501,8 +489,6 @@ mla_status mla_epilogue_launch(
   size_t smem = 0;
   if (plan.mode == MLA_MODE_SPLIT) {
     fn = mla::kSplitKernels[k];
-  } else if (plan.mode == MLA_MODE_TOKEN) {
-    fn = mla::kTokenKernels[k];
   } else {
     s = mla::rows_kernel(k, plan.threads_per_block / 32, &fn, &smem);
     if (s != MLA_OK) return s;

@@ -11,8 +11,8 @@ namespace mla {
 
 // Upper limits (and defaults) of the tuning knobs mla_epilogue_set_tuning
 // clamps to.
-constexpr int kRowsMaxBlocksPerSm = 5;  // resident blocks per SM the kernel is compiled for
-constexpr int kRowsMaxWarps = 8;        // warps per block (each with its own 4.5 KB row ring)
+constexpr int kRowsMaxBlocksPerSm = 5;  // resident blocks per SM the kernel is compiled for (48 registers)
+constexpr int kRowsMaxWarps = 8;        // warps per block
 constexpr int kRowsDefaultWarps = 8;
 
 // Grid and block of a ROWS launch over `rows` rows.

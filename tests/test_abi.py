@@ -79,7 +79,7 @@ def _call(**kw):
     (dict(flags=1 << 31), E.MLA_ERR_UNSUPPORTED),
     (dict(flags=128), E.MLA_ERR_UNSUPPORTED),
     (dict(flags=E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS), E.MLA_ERR_INVALID_ARG),
-    (dict(flags=E.MLA_FLAG_FORCE_TOKEN | E.MLA_FLAG_FORCE_ROWS), E.MLA_ERR_INVALID_ARG),
+    (dict(flags=64), E.MLA_ERR_UNSUPPORTED),
     (dict(T=-1), E.MLA_ERR_INVALID_ARG),
     (dict(H=0), E.MLA_ERR_INVALID_ARG),
     (dict(H=65537), E.MLA_ERR_INVALID_ARG),
@@ -135,10 +135,11 @@ def test_size_one_dimensions_skip_stride_checks(lib):
 
 def test_plan_modes_and_grids(lib):
     t = E.mla_epilogue_get_tuning()
+    assert t.split_threads_per_block == 0  # automatic block size
     p = E.mla_epilogue_plan(64, 16, 0, sm_count=148)
-    assert p.mode == E.MLA_MODE_SPLIT and p.threads_per_block == 68 * p.rows_per_block
-    assert p.rows_per_block == t.split_rows_per_block
-    assert p.blocks == -(-64 * 17 // p.rows_per_block)
+    assert p.mode == E.MLA_MODE_SPLIT and p.rows_per_block == 0
+    # 68 threads per row over about one block per SM: 64 * 17 * 68 / 148 -> 512
+    assert p.threads_per_block == 512 and p.blocks == -(-64 * 17 * 68 // 512) <= 148
     # the default split threshold counts rows: 4608 = 271 tokens x 17 rows, rounded up
     assert t.split_max_rows == 4608
     assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
@@ -147,28 +148,27 @@ def test_plan_modes_and_grids(lib):
     assert E.mla_epilogue_plan(32, 128, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
     assert E.mla_epilogue_plan(36, 128, 0, sm_count=148).mode == E.MLA_MODE_ROWS
     p = E.mla_epilogue_plan(300, 16, 0, sm_count=148)
-    assert p.mode == E.MLA_MODE_ROWS and p.threads_per_block % 32 == 0
+    assert p.mode == E.MLA_MODE_ROWS and p.threads_per_block % 32 == 0 and p.rows_per_block == 1
     assert p.blocks <= 148 * t.rows_blocks_per_sm
     assert E.mla_epilogue_plan(1, 16, E.MLA_FLAG_FORCE_ROWS, sm_count=148).mode == E.MLA_MODE_ROWS
-    assert E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148).mode == E.MLA_MODE_SPLIT
-    assert E.mla_epilogue_plan(9, 16, E.MLA_FLAG_FORCE_TOKEN, sm_count=148).mode == E.MLA_MODE_TOKEN
+    big = E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148)
+    assert big.mode == E.MLA_MODE_SPLIT and big.threads_per_block == 1024
+    assert big.blocks == -(-8192 * 17 * 68 // 1024)
     with pytest.raises(E.MlaError):
         E.mla_epilogue_plan(0, 16, 0, sm_count=148)
-    for bad in (E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS, E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_TOKEN,
-                E.MLA_FLAG_FORCE_ROWS | E.MLA_FLAG_FORCE_TOKEN):
-        with pytest.raises(E.MlaError):
-            E.mla_epilogue_plan(4, 16, bad, sm_count=148)
+    with pytest.raises(E.MlaError):
+        E.mla_epilogue_plan(4, 16, E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS, sm_count=148)
 
 
-@pytest.mark.parametrize("H,blocks", [(1, 1), (16, 1), (27, 1), (28, 2), (128, 5)])
-def test_single_token_plan_puts_the_token_in_one_block(lib, H, blocks):
-    """T == 1 takes MLA_MODE_TOKEN: 36 threads per row, every row of the
-    token in one block while H + 1 <= 28 rows fit in 1024 threads."""
-    p = E.mla_epilogue_plan(1, H, E.MLA_FLAG_ROPE, sm_count=148)
-    assert p.mode == E.MLA_MODE_TOKEN
-    assert p.rows_per_block == min(H + 1, 28) and p.threads_per_block == 36 * p.rows_per_block
-    assert p.blocks == blocks and p.blocks * p.rows_per_block >= H + 1
-    assert E.mla_epilogue_plan(2, H, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
+@pytest.mark.parametrize("T,H,threads,blocks", [(1, 16, 32, 37), (1, 1, 32, 5), (1, 128, 64, 138), (4, 16, 32, 145),
+                                                (16, 16, 128, 145), (2, 16, 32, 73)])
+def test_decode_sizes_spread_over_the_sms(lib, T, H, threads, blocks):
+    """At decode sizes the plan gives about one block per SM, so a single
+    token's rows run on as many SMs as possible (one-warp blocks)."""
+    p = E.mla_epilogue_plan(T, H, E.MLA_FLAG_ROPE, sm_count=148)
+    assert p.mode == E.MLA_MODE_SPLIT
+    assert (p.threads_per_block, p.blocks) == (threads, blocks)
+    assert p.blocks * p.threads_per_block >= T * (H + 1) * 68
 
 
 def test_tuning_moves_the_threshold_and_clamps(lib):
@@ -177,17 +177,20 @@ def test_tuning_moves_the_threshold_and_clamps(lib):
         E.mla_epilogue_set_tuning(split_max_rows=64 * 17)
         assert E.mla_epilogue_plan(64, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
         assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_ROWS
-        E.mla_epilogue_set_tuning(split_rows_per_block=99, rows_warps_per_block=99, rows_blocks_per_sm=99)
+        E.mla_epilogue_set_tuning(split_threads_per_block=5000, rows_warps_per_block=99, rows_blocks_per_sm=99)
         t = E.mla_epilogue_get_tuning()
-        assert t.split_rows_per_block == 15 and 68 * t.split_rows_per_block <= 1024
+        assert t.split_threads_per_block == 1024
         assert t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 5
-        E.mla_epilogue_set_tuning(split_rows_per_block=3)
+        E.mla_epilogue_set_tuning(split_threads_per_block=200)  # rounded up to whole warps
         p = E.mla_epilogue_plan(5, 16, 0, sm_count=148)
-        assert p.rows_per_block == 3 and p.threads_per_block == 204 and p.blocks == 29
+        assert p.threads_per_block == 224 and p.blocks == -(-5 * 17 * 68 // 224)
         E.mla_epilogue_set_tuning()  # all zero: unchanged
         assert E.mla_epilogue_get_tuning().split_max_rows == 64 * 17
+        assert E.mla_epilogue_get_tuning().split_threads_per_block == 224
+        E.mla_epilogue_set_tuning(split_threads_per_block=-1)  # back to automatic
+        assert E.mla_epilogue_get_tuning().split_threads_per_block == 0
     finally:
-        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_rows_per_block,
+        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_threads_per_block or -1,
                                   old.rows_warps_per_block, old.rows_blocks_per_sm)
 
 

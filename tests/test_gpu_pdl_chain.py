@@ -53,7 +53,7 @@ def _expected_scores(w, q, cache):
     return prod.sum(-1).reshape(-1), prod.abs().sum(-1).reshape(-1)
 
 
-@pytest.mark.parametrize("force", [0, E.MLA_FLAG_FORCE_SPLIT, E.MLA_FLAG_FORCE_ROWS, E.MLA_FLAG_FORCE_TOKEN])
+@pytest.mark.parametrize("force", [0, E.MLA_FLAG_FORCE_SPLIT, E.MLA_FLAG_FORCE_ROWS])
 @pytest.mark.parametrize("T,flags", [(7, W.FLAG_ROPE), (64, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8),
                                      (300, W.FLAG_ROPE | W.FLAG_KV_FP8), (1500, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8)])
 def test_consumer_behind_epilogue_sees_every_store(force, T, flags):
