@@ -467,7 +467,7 @@ def standalone(hx, ds, device, calls, reps, peak):
 
 
 def mode_name(E, plan):
-    return {E.MLA_MODE_SPLIT: "split", E.MLA_MODE_ROWS: "rows", E.MLA_MODE_TOKEN: "token"}[plan.mode]
+    return {E.MLA_MODE_SPLIT: "split", E.MLA_MODE_ROWS: "rows"}[plan.mode]
 
 
 def decode_floors(hx, device, peak, calls=200, reps=7):
