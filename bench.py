@@ -472,13 +472,18 @@ def mode_name(E, plan):
 
 def decode_floors(hx, device, peak, calls=200, reps=7):
     """T = 1 .. 64 (the decode sweep workload: H=16, RoPE, e4m3): standalone
-    with cold inputs, and behind the producer with PDL against the floor of
-    a dependent launch."""
+    with cold inputs (`floor_ratio`: against an empty kernel of the same
+    grid), and behind the producer with PDL: `floor_ratio_behind_producer`
+    is the epilogue's increment over the producer against the increment of
+    an empty dependent that waits, `increment_over_launch_floor` the same
+    increment against one bare launch of an empty kernel."""
     out = []
     for T in DECODE_T:
         ds = DeviceSets(f"decode_sweep_t{T}_h16_rope_fp8")
         row = standalone(hx, ds, device, calls, reps, peak)
         row.update(behind_producer(hx, ds, device, calls, reps))
+        # the epilogue's cost behind the producer against one bare launch
+        row["increment_over_launch_floor"] = round(row["epilogue_increment_pdl_us"] / row["launch_floor_us"], 3)
         out.append(row)
         del ds
         torch.cuda.empty_cache()

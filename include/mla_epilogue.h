@@ -77,8 +77,7 @@ typedef enum mla_status {
 #define MLA_MODE_SPLIT 1 /* small T: 68 threads per 576-wide row, 64 with one 16-byte nope chunk each and 4 with
                             eight RoPE pairs each (16-byte loads); threads map to rows by their index in the grid
                             and blocks are sized to about one per SM (one-warp blocks for a single token) */
-#define MLA_MODE_ROWS  2 /* large T: one warp per row, grid-stride, slot and position loaded one row ahead;
-                            grid sized to the resident blocks */
+#define MLA_MODE_ROWS  2 /* large T: one warp per row, grid-stride, grid sized to the resident blocks */
 
 /*
  * mla_epilogue_launch -- the whole epilogue in one kernel launch.
@@ -182,8 +181,8 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  *                        a negative value restores the default
  *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8 (default 8)
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
- *                        5, the number the kernel's register cap keeps resident
- *                        (default 5)
+ *                        the number the kernel's register cap keeps resident (6 with
+ *                        an e4m3 output, 5 without; default: that number)
  * Larger values are clamped to those limits; 0 keeps the current setting.
  */
 typedef struct mla_tuning {

@@ -15,9 +15,10 @@
 //     and 32+8j..32+8j+7, so one thread holds both members of its 8 RoPE
 //     pairs (i, i+32) and rotates them without shuffles, with 16-byte loads
 //     and 16-byte (bf16) or 8-byte (e4m3) stores.  Threads map to work by
-//     their index in the grid: the first 64 * rows threads are the nope
-//     threads of all rows, the next 4 * rows the pe threads (eight rows per
-//     warp), so every warp has one role and the block size is free.  At
+//     their index in the grid: the first 4 * rows threads are the pe threads
+//     of all rows (eight rows per warp; their position -> table chain is the
+//     longest, and blocks start in index order), the next 64 * rows the nope
+//     threads, so every warp has one role and the block size is free.  At
 //     decode sizes the latency is lowest when the work is spread over as
 //     many SMs as there are (measured on B200: one 17-row token in 37
 //     one-warp blocks is about 0.9 us faster than in one to three blocks),
@@ -240,12 +241,13 @@ __device__ __forceinline__ void small_query_row(const Args& a, int64_t q, bool p
 
 template <bool QF8, bool KVF8, bool ROPE>
 __global__ void __launch_bounds__(kSmallMaxThreads) mla_epilogue_small_kernel(const Args a) {
-  // thread -> (row, part) by its index in the grid: nope threads of all rows
-  // first (64 per row), then pe threads (4 per row)
+  // thread -> (row, part) by its index in the grid: the pe threads of all
+  // rows first (4 per row: their position -> table chain is the longest, and
+  // blocks are dispatched in index order), then the nope threads (64 per row)
   const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nope_threads = 64 * a.rows;
-  const bool pe = gt >= nope_threads;
-  const int64_t u = pe ? gt - nope_threads : gt;
+  const int64_t pe_threads = 4 * a.rows;
+  const bool pe = gt < pe_threads;
+  const int64_t u = pe ? gt : gt - pe_threads;
   const int64_t g = pe ? (u >> 2) : (u >> 6);
   const int part = static_cast<int>(pe ? (u & 3) : (u & 63));
   if (g < a.rows) {

@@ -6,9 +6,9 @@
 // order (vLLM PR #54896 report, 实现拆解 items 1-3).  Warp w of the grid
 // takes rows w, w + W, w + 2W, ... (W = all warps of the grid), so all warps
 // walk one window of memory together.  Lane l moves nope chunks l and l + 32
-// (16 bytes each) and rotates pe pair (l, l + 32).  A row's slot and
-// position are loaded one row ahead, so the row's data loads and its table
-// row go out together: one memory round trip per row, not two.
+// (16 bytes each) and rotates pe pair (l, l + 32): the e4m3 arithmetic of a
+// row is spread over all 32 lanes, which matters because the e4m3 kernel is
+// bound by instruction issue as much as by memory (measured on B200).
 //
 // Query rows execute griddepcontrol.wait once, before their first read of
 // q_nope / q_pe (the upstream kernel writes them); cache rows, slots,
@@ -26,11 +26,31 @@
 namespace mla {
 namespace rows {
 
-// Rotation of pair `i` of a row: (cos, sin) from the table row of its token's position.
+// Resident 256-thread blocks per SM the kernel is compiled for: 5 (a
+// 48-register cap) for bf16 outputs; 6 (40 registers) when an output is
+// e4m3, whose arithmetic leaves the kernel short of memory parallelism at 5
+// (measured on B200: 0.75 -> 0.78 of copy bandwidth for T=8192, H=16; the
+// bf16 variants lose at 6).
+constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 6 : 5; }
+static_assert(rows_blocks_per_sm(true, true) <= kRowsMaxBlocksPerSm, "tuning limit covers the resident count");
+
+// Rotation of pair `i` for token t: (cos, sin) from the table row of its position.
 struct Rot {
   float c, s;
   bool on;
 };
+
+__device__ __forceinline__ Rot load_rotation(const Args& a, int64_t t, int i) {
+  Rot r{1.0f, 0.0f, false};
+  const int64_t pos = __ldg(a.positions + t);
+  if (pos >= 0 && pos < a.rope_rows) {
+    const float* row = a.cos_sin + pos * kPe;
+    r.c = __ldg(row + i);
+    r.s = __ldg(row + kHalfPe + i);
+    r.on = true;
+  }
+  return r;
+}
 
 template <bool FP8, bool FAST>
 __device__ __forceinline__ void store_nope(uint8_t* dst, int chunk, const uint4 v, const Divisor& d) {
@@ -80,76 +100,54 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* pe, int i) {
 // rows kernel: one warp per row, grid-stride over rows
 // ------------------------------------------------------------------------------------
 
-// A row's cache slot (cache rows) and token position, loaded one row ahead.
-struct Pre {
-  int64_t slot;
-  int32_t pos;
-};
-
-template <bool ROPE>
-__device__ __forceinline__ Pre prefetch(const Args& a, int64_t g) {
-  Pre p{-1, -1};
-  if (g < a.rows) {
-    const int64_t t = g < a.T ? g : div_heads(a, g - a.T);
-    if (g < a.T) p.slot = __ldg(a.slots + t);
-    if constexpr (ROPE) p.pos = __ldg(a.positions + t);
-  }
-  return p;
-}
-
 template <bool QF8, bool KVF8, bool ROPE, bool FAST>
 __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, const Divisor& dk) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   bool waited = false;
-  Pre nx = prefetch<ROPE>(a, wid);
+
   for (int64_t g = wid; g < a.rows; g += warps) {
-    const Pre cur = nx;
-    nx = prefetch<ROPE>(a, g + warps);
+    // 1. addresses, slot and rotation: nothing here depends on the upstream kernel
     const bool is_cache = g < a.T;
-    int64_t q = 0, t;
+    int64_t t;
     const uint16_t* nope;
     const uint16_t* pe;
+    uint8_t* dst = nullptr;
     if (is_cache) {
       t = g;
       nope = a.kv_c + t * a.kv_st;
       pe = a.k_pe + t * a.kp_st;
+      const int64_t slot = __ldg(a.slots + t);
+      if (slot >= 0 && slot < a.cache_rows) {
+        dst = a.cache + slot * (KVF8 ? kRow : 2 * kRow);
+      } else if (slot >= a.cache_rows && lane == 0) {
+        report(a.status, MLA_STATUS_SLOT_RANGE);
+      }
     } else {
-      q = g - a.T;
+      const int64_t q = g - a.T;
       t = div_heads(a, q);
       const int64_t h = q - t * a.H;
       nope = a.q_nope + t * a.qn_st + h * a.qn_sh;
       pe = a.q_pe + t * a.qp_st + h * a.qp_sh;
-      if (!waited) {  // query rows read what the upstream kernel wrote: wait for it once
-        pdl_wait();
-        waited = true;
-      }
+      dst = a.q_out + q * (QF8 ? kRow : 2 * kRow);
     }
-    // the row's loads and its rotation (position known from the row before): one round trip
+    Rot rot{1.0f, 0.0f, false};
+    if constexpr (ROPE) {
+      rot = load_rotation(a, t, lane);
+      if (is_cache && lane == 0 && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
+    }
+
+    // 2. query rows read what the upstream kernel wrote: wait for it once
+    if (!is_cache && !waited) {
+      pdl_wait();
+      waited = true;
+    }
+
+    // 3. the row's loads, then 4. convert and store
     const uint4 n0 = ld_chunk(nope, lane);
     const uint4 n1 = ld_chunk(nope, lane + 32);
     const uint32_t p = ld_pair(pe, lane);
-    Rot rot{1.0f, 0.0f, false};
-    if constexpr (ROPE) {
-      if (cur.pos >= 0 && cur.pos < a.rope_rows) {
-        const float* row = a.cos_sin + static_cast<int64_t>(cur.pos) * kPe;
-        rot.c = __ldg(row + lane);
-        rot.s = __ldg(row + kHalfPe + lane);
-        rot.on = true;
-      }
-    }
-    uint8_t* dst = nullptr;
-    if (is_cache) {
-      if (cur.slot >= 0 && cur.slot < a.cache_rows) {
-        dst = a.cache + cur.slot * (KVF8 ? kRow : 2 * kRow);
-      } else if (cur.slot >= a.cache_rows && lane == 0) {
-        report(a.status, MLA_STATUS_SLOT_RANGE);
-      }
-      if (ROPE && !rot.on && lane == 0) report(a.status, MLA_STATUS_POS_RANGE);
-    } else {
-      dst = a.q_out + q * (QF8 ? kRow : 2 * kRow);
-    }
     if (dst == nullptr) continue;
     if (is_cache) {
       store_nope<KVF8, FAST>(dst, lane, n0, dk);
@@ -164,7 +162,7 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
 }
 
 template <bool QF8, bool KVF8, bool ROPE>
-__global__ void __launch_bounds__(32 * kRowsMaxWarps, kRowsMaxBlocksPerSm) mla_epilogue_rows_kernel(const Args a) {
+__global__ void __launch_bounds__(32 * kRowsMaxWarps, rows_blocks_per_sm(QF8, KVF8)) mla_epilogue_rows_kernel(const Args a) {
   // scales are read before any wait; the whole body takes the corrected-
   // reciprocal quotient unless a scale is outside [2^-64, 2^64]
   Divisor dq{}, dk{};
@@ -190,11 +188,12 @@ const void* const kKernels[8] = {kernel_for<0>(), kernel_for<1>(), kernel_for<2>
 
 }  // namespace rows
 
-void rows_plan(int64_t rows, bool, bool, int32_t sm_count, int32_t blocks_per_sm, int32_t warps_per_block,
+void rows_plan(int64_t rows, bool qf8, bool kvf8, int32_t sm_count, int32_t blocks_per_sm, int32_t warps_per_block,
                mla_plan* p) {
   const int32_t w = warps_per_block < kRowsMaxWarps ? warps_per_block : kRowsMaxWarps;
   const int64_t need = (rows + w - 1) / w;
-  const int32_t per_sm = blocks_per_sm < kRowsMaxBlocksPerSm ? blocks_per_sm : kRowsMaxBlocksPerSm;
+  const int32_t resident = rows::rows_blocks_per_sm(qf8, kvf8);
+  const int32_t per_sm = blocks_per_sm < resident ? blocks_per_sm : resident;
   const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
   p->mode = MLA_MODE_ROWS;
   p->rows_per_block = 1;

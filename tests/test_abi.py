@@ -180,7 +180,7 @@ def test_tuning_moves_the_threshold_and_clamps(lib):
         E.mla_epilogue_set_tuning(split_threads_per_block=5000, rows_warps_per_block=99, rows_blocks_per_sm=99)
         t = E.mla_epilogue_get_tuning()
         assert t.split_threads_per_block == 1024
-        assert t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 5
+        assert t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 6
         E.mla_epilogue_set_tuning(split_threads_per_block=200)  # rounded up to whole warps
         p = E.mla_epilogue_plan(5, 16, 0, sm_count=148)
         assert p.threads_per_block == 224 and p.blocks == -(-5 * 17 * 68 // 224)
