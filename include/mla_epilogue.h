@@ -74,9 +74,9 @@ typedef enum mla_status {
                                     out; the kernel returns instead of hanging */
 
 /* Kernel choice (mla_plan.mode). */
-#define MLA_MODE_SPLIT 1 /* small T: 68 threads per 576-wide row, 64 with one 16-byte nope chunk each and 4 with
-                            eight RoPE pairs each (16-byte loads); threads map to rows by their index in the grid
-                            and blocks are sized to about one per SM (one-warp blocks for a single token) */
+#define MLA_MODE_SPLIT 1 /* small T: three warps per 576-wide row (two move 16-byte nope chunks, one rotates the
+                            32 RoPE pairs, one per lane); rows_per_block rows per block, ceil(rows / SMs) unless
+                            tuned, so a single token's rows run one per SM */
 #define MLA_MODE_ROWS  2 /* large T: one warp per row, grid-stride, grid sized to the resident blocks */
 
 /*
@@ -160,8 +160,8 @@ typedef struct mla_plan {
   int32_t mode;              /* MLA_MODE_SPLIT or MLA_MODE_ROWS */
   int32_t threads_per_block;
   int64_t blocks;
-  int32_t rows_per_block;    /* ROWS: 1 (one row per warp at a time); SPLIT: 0 (rows spread over blocks by
-                                thread index, 68 threads a row) */
+  int32_t rows_per_block;    /* SPLIT: rows one block covers (96 threads each); ROWS: 1 (one row per warp at a
+                                time) */
   int32_t sm_count;
 } mla_plan;
 
@@ -176,9 +176,9 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  * (T * (H + 1)) whatever H is (measured for H = 8, 16, 32, 128), so the
  * default threshold counts rows, not tokens.
  *   split_max_rows       T * (H + 1) at or below which MLA_MODE_SPLIT is used (default 4608)
- *   split_threads_per_block threads per block in MLA_MODE_SPLIT, rounded up to a multiple of
- *                        32, at most 1024; 0 (default) sizes blocks to about one per SM;
- *                        a negative value restores the default
+ *   split_rows_per_block rows per block in MLA_MODE_SPLIT (block = 96 * this), at most
+ *                        10; 0 (default) takes ceil(rows / SMs); a negative value
+ *                        restores the default
  *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8 (default 8)
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
  *                        the number the kernel's register cap keeps resident (6 with
@@ -187,7 +187,7 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  */
 typedef struct mla_tuning {
   int64_t split_max_rows;
-  int32_t split_threads_per_block;
+  int32_t split_rows_per_block;
   int32_t rows_warps_per_block;
   int32_t rows_blocks_per_sm;
 } mla_tuning;

@@ -10,21 +10,15 @@
 // bound by launch and memory latency, at large T by HBM bandwidth; there is
 // no contraction and no tensor-core work.  Three launch modes:
 //
-//   SPLIT (small T): every row gets 68 threads.  64 of them move one 16-byte
-//     nope chunk each (8 values); 4 of them each own the pe octets 8j..8j+7
-//     and 32+8j..32+8j+7, so one thread holds both members of its 8 RoPE
-//     pairs (i, i+32) and rotates them without shuffles, with 16-byte loads
-//     and 16-byte (bf16) or 8-byte (e4m3) stores.  Threads map to work by
-//     their index in the grid: the first 4 * rows threads are the pe threads
-//     of all rows (eight rows per warp; their position -> table chain is the
-//     longest, and blocks start in index order), the next 64 * rows the nope
-//     threads, so every warp has one role and the block size is free.  At
-//     decode sizes the latency is lowest when the work is spread over as
-//     many SMs as there are (measured on B200: one 17-row token in 37
-//     one-warp blocks is about 0.9 us faster than in one to three blocks),
-//     so the plan sizes blocks to give about one block per SM; for T = 1
-//     that is one-warp blocks (the num_tokens == 1 case of PR #53526,
-//     关联脉络).
+//   SPLIT (small T): every row gets three warps, as the page's SPLIT=3 path
+//     does.  Warps 0 and 1 move the 64 nope chunks (16 bytes, 8 values, one
+//     chunk per lane); warp 2 rotates the 64 pe values as 32 RoPE pairs
+//     (i, i+32), one pair per lane, so the rotation needs no shuffles and
+//     each thread's chain of dependent work stays short.  A block holds R
+//     rows; at decode sizes latency falls as the rows spread over more SMs
+//     (measured on B200), so the plan takes R = ceil(rows / SMs): one row per
+//     block for a single token (the num_tokens == 1 case of PR #53526,
+//     关联脉络), more rows per block only once every SM has one.
 //   ROWS (large T): mla_rows.cu.
 //
 // In SPLIT every thread computes its addresses and loads its slot,
@@ -46,118 +40,8 @@
 
 namespace mla {
 
-constexpr int kSmallMaxThreads = 1024;
-constexpr int kSmallThreadsPerRow = 68;  // 64 nope threads + 4 pe threads
-
-// Nope chunk `chunk` (8 values) of a row: 16 bytes in, 16 (bf16) or 8 (e4m3) out.
-template <bool FP8, bool FAST>
-__device__ __forceinline__ void store_nope(uint8_t* dst, int chunk, const uint4 v, const Divisor& d) {
-  if constexpr (FP8) {
-    *reinterpret_cast<uint2*>(dst + chunk * 8) = chunk_to_e4m3<FAST>(v, d);
-  } else {
-    *reinterpret_cast<uint4*>(dst + chunk * 16) = v;
-  }
-}
-
-// Rotation of the pairs 8j .. 8j+7 of token t: cos and sin from the table row
-// of its position, or `on` false when RoPE is off or the position is out of
-// range.
-struct Rot8 {
-  float c[8], s[8];
-  bool on;
-};
-
-template <bool ROPE>
-__device__ __forceinline__ Rot8 load_rot8(const Args& a, int64_t t, int j) {
-  Rot8 r;
-  r.on = false;
-  if constexpr (ROPE) {
-    const int64_t pos = __ldg(a.positions + t);
-    if (pos >= 0 && pos < a.rope_rows) {
-      const float* row = a.cos_sin + pos * kPe + 8 * j;
-      if (a.tab_vec) {
-        const float4 c0 = __ldg(reinterpret_cast<const float4*>(row));
-        const float4 c1 = __ldg(reinterpret_cast<const float4*>(row) + 1);
-        const float4 s0 = __ldg(reinterpret_cast<const float4*>(row + kHalfPe));
-        const float4 s1 = __ldg(reinterpret_cast<const float4*>(row + kHalfPe) + 1);
-        r.c[0] = c0.x; r.c[1] = c0.y; r.c[2] = c0.z; r.c[3] = c0.w;
-        r.c[4] = c1.x; r.c[5] = c1.y; r.c[6] = c1.z; r.c[7] = c1.w;
-        r.s[0] = s0.x; r.s[1] = s0.y; r.s[2] = s0.z; r.s[3] = s0.w;
-        r.s[4] = s1.x; r.s[5] = s1.y; r.s[6] = s1.z; r.s[7] = s1.w;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          r.c[k] = __ldg(row + k);
-          r.s[k] = __ldg(row + kHalfPe + k);
-        }
-      }
-      r.on = true;
-    }
-  }
-  return r;
-}
-
-// pe values 8j .. 8j+7 (`lo`) and 32+8j .. 32+8j+7 (`hi`) of one row as bf16
-// words (value 2k in the low half of word k): two 16-byte loads when the row
-// is 16-byte aligned, else sixteen 2-byte loads.
-__device__ __forceinline__ void load_pe8(const uint16_t* pe, int j, bool vec, uint4& lo, uint4& hi) {
-  if (vec) {
-    lo = ld_cg16(pe + 8 * j);
-    hi = ld_cg16(pe + kHalfPe + 8 * j);
-  } else {
-    uint32_t w[8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      w[k] = static_cast<uint32_t>(__ldcg(pe + 8 * j + 2 * k)) |
-             (static_cast<uint32_t>(__ldcg(pe + 8 * j + 2 * k + 1)) << 16);
-      w[4 + k] = static_cast<uint32_t>(__ldcg(pe + kHalfPe + 8 * j + 2 * k)) |
-                 (static_cast<uint32_t>(__ldcg(pe + kHalfPe + 8 * j + 2 * k + 1)) << 16);
-    }
-    lo = make_uint4(w[0], w[1], w[2], w[3]);
-    hi = make_uint4(w[4], w[5], w[6], w[7]);
-  }
-}
-
-// The 8 RoPE pairs (8j + k, 32 + 8j + k), k < 8, of a row: rotate in fp32, encode,
-// store 2 x 16 bytes (bf16) or 2 x 8 bytes (e4m3).
-template <bool FP8, bool ROPE, bool FAST>
-__device__ __forceinline__ void store_pe8(uint8_t* row, int j, const uint4 lo, const uint4 hi, const Rot8& r,
-                                          const Divisor& d) {
-  const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
-  const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
-  float ya[8], yb[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float a = (k & 1) ? bf16_hi(wl[k >> 1]) : bf16_lo(wl[k >> 1]);
-    const float b = (k & 1) ? bf16_hi(wh[k >> 1]) : bf16_lo(wh[k >> 1]);
-    ya[k] = a;
-    yb[k] = b;
-    if (ROPE && r.on) rope_pair(a, b, r.c[k], r.s[k], ya[k], yb[k]);
-  }
-  if constexpr (FP8) {
-    uint2 oa, ob;
-    oa.x = e4m3x2_of_f32<FAST>(ya[0], ya[1], d) | (e4m3x2_of_f32<FAST>(ya[2], ya[3], d) << 16);
-    oa.y = e4m3x2_of_f32<FAST>(ya[4], ya[5], d) | (e4m3x2_of_f32<FAST>(ya[6], ya[7], d) << 16);
-    ob.x = e4m3x2_of_f32<FAST>(yb[0], yb[1], d) | (e4m3x2_of_f32<FAST>(yb[2], yb[3], d) << 16);
-    ob.y = e4m3x2_of_f32<FAST>(yb[4], yb[5], d) | (e4m3x2_of_f32<FAST>(yb[6], yb[7], d) << 16);
-    *reinterpret_cast<uint2*>(row + kNope + 8 * j) = oa;
-    *reinterpret_cast<uint2*>(row + kNope + kHalfPe + 8 * j) = ob;
-  } else {
-    uint4 oa = lo, ob = hi;  // unrotated values keep their bits (NaN payloads included)
-    if (ROPE && r.on) {
-      oa = make_uint4(pack_bf16x2(ya[0], ya[1]), pack_bf16x2(ya[2], ya[3]), pack_bf16x2(ya[4], ya[5]),
-                      pack_bf16x2(ya[6], ya[7]));
-      ob = make_uint4(pack_bf16x2(yb[0], yb[1]), pack_bf16x2(yb[2], yb[3]), pack_bf16x2(yb[4], yb[5]),
-                      pack_bf16x2(yb[6], yb[7]));
-    }
-    *reinterpret_cast<uint4*>(row + 2 * (kNope + 8 * j)) = oa;
-    *reinterpret_cast<uint4*>(row + 2 * (kNope + kHalfPe + 8 * j)) = ob;
-  }
-}
-
-// ------------------------------------------------------------------------------------
-// small-batch kernel
-// ------------------------------------------------------------------------------------
+constexpr int kSplitThreadsPerRow = 96;  // three warps
+constexpr int kSplitMaxRowsPerBlock = 10;  // 960 threads
 
 // A row's e4m3 scale: its load is issued with the row's other loads and the
 // divisor is made only when the stores need it, so the scale adds no step
@@ -168,108 +52,98 @@ __device__ __forceinline__ float scale_of(const float* scale) {
   return 1.0f;
 }
 
-template <bool FP8>
-__device__ __forceinline__ Divisor divisor_from(float scale) {
+// The stores of one lane's slice of a row (nope chunk `chunk` for parts 0
+// and 1, pe pair `lane` for part 2), on the quotient path the scale selects:
+// the corrected reciprocal unless the scale is outside [2^-64, 2^64].
+template <bool FP8, bool ROPE>
+__device__ __forceinline__ void split_store(uint8_t* dst, int part, int lane, const uint4& v, uint32_t pe,
+                                            const Rot& rot, float scale) {
   Divisor d{};
   d.fast = true;
   if constexpr (FP8) d = make_divisor(scale);
-  return d;
-}
-
-// Stores of one thread's share of a row, the quotient path chosen from the
-// scale: the corrected reciprocal unless the scale is outside [2^-64, 2^64].
-template <bool FP8, bool ROPE>
-__device__ __forceinline__ void store_part(uint8_t* dst, bool pe, int part, const uint4& v, const uint4& lo,
-                                           const uint4& hi, const Rot8& rot, float scale) {
-  const Divisor d = divisor_from<FP8>(scale);
   if (!FP8 || d.fast) {
-    if (!pe) {
-      store_nope<FP8, true>(dst, part, v, d);
+    if (part < 2) {
+      store_nope<FP8, true>(dst, part * 32 + lane, v, d);
     } else {
-      store_pe8<FP8, ROPE, true>(dst, part, lo, hi, rot, d);
+      store_pe<FP8, ROPE, true>(dst, lane, pe, rot, d);
     }
   } else {
-    if (!pe) {
-      store_nope<FP8, false>(dst, part, v, d);
+    if (part < 2) {
+      store_nope<FP8, false>(dst, part * 32 + lane, v, d);
     } else {
-      store_pe8<FP8, ROPE, false>(dst, part, lo, hi, rot, d);
+      store_pe<FP8, ROPE, false>(dst, lane, pe, rot, d);
     }
   }
 }
 
 template <bool FP8, bool ROPE>
-__device__ __forceinline__ void small_cache_row(const Args& a, int64_t t, bool pe, int part) {
+__device__ __forceinline__ void split_cache_row(const Args& a, int64_t t, int part, int lane) {
   const float scale = scale_of<FP8>(a.kv_scale);
   const int64_t slot = __ldg(a.slots + t);
-  uint4 v = make_uint4(0, 0, 0, 0), lo = v, hi = v;
-  Rot8 rot;
-  rot.on = false;
-  if (!pe) {
-    v = ld_cg16(a.kv_c + t * a.kv_st + 8 * part);
+  uint4 v = make_uint4(0, 0, 0, 0);
+  uint32_t pe = 0;
+  Rot rot{1.0f, 0.0f, false};
+  if (part < 2) {
+    v = ld_chunk(a.kv_c + t * a.kv_st, part * 32 + lane);
   } else {
-    rot = load_rot8<ROPE>(a, t, part);
-    load_pe8(a.k_pe + t * a.kp_st, part, a.kpe_vec != 0, lo, hi);
+    pe = ld_pair(a.k_pe + t * a.kp_st, lane);
+    if constexpr (ROPE) rot = load_rotation(a, t, lane);
   }
-  const bool in_range = slot >= 0 && slot < a.cache_rows;
-  if (part == 0) {
-    if (!pe && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
-    if (ROPE && pe && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
+  if (lane == 0) {
+    if (part == 0 && slot >= a.cache_rows) report(a.status, MLA_STATUS_SLOT_RANGE);
+    if (ROPE && part == 2 && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
   }
-  if (in_range) store_part<FP8, ROPE>(a.cache + slot * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
+  if (slot >= 0 && slot < a.cache_rows)
+    split_store<FP8, ROPE>(a.cache + slot * (FP8 ? kRow : 2 * kRow), part, lane, v, pe, rot, scale);
 }
 
 template <bool FP8, bool ROPE>
-__device__ __forceinline__ void small_query_row(const Args& a, int64_t q, bool pe, int part) {
+__device__ __forceinline__ void split_query_row(const Args& a, int64_t q, int part, int lane) {
   const float scale = scale_of<FP8>(a.q_scale);
   const int64_t t = div_heads(a, q);
   const int64_t h = q - t * a.H;
-  uint4 v = make_uint4(0, 0, 0, 0), lo = v, hi = v;
-  Rot8 rot;
-  rot.on = false;
-  if (!pe) {
-    const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh + 8 * part;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  uint32_t pe = 0;
+  Rot rot{1.0f, 0.0f, false};
+  if (part < 2) {
+    const uint16_t* src = a.q_nope + t * a.qn_st + h * a.qn_sh;
     pdl_wait();
-    v = ld_cg16(src);
+    v = ld_chunk(src, part * 32 + lane);
   } else {
     const uint16_t* src = a.q_pe + t * a.qp_st + h * a.qp_sh;
-    rot = load_rot8<ROPE>(a, t, part);
+    if constexpr (ROPE) rot = load_rotation(a, t, lane);
     pdl_wait();
-    load_pe8(src, part, a.qpe_vec != 0, lo, hi);
+    pe = ld_pair(src, lane);
   }
-  store_part<FP8, ROPE>(a.q_out + q * (FP8 ? kRow : 2 * kRow), pe, part, v, lo, hi, rot, scale);
+  split_store<FP8, ROPE>(a.q_out + q * (FP8 ? kRow : 2 * kRow), part, lane, v, pe, rot, scale);
 }
 
 template <bool QF8, bool KVF8, bool ROPE>
-__global__ void __launch_bounds__(kSmallMaxThreads) mla_epilogue_small_kernel(const Args a) {
-  // thread -> (row, part) by its index in the grid: the pe threads of all
-  // rows first (4 per row: their position -> table chain is the longest, and
-  // blocks are dispatched in index order), then the nope threads (64 per row)
-  const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t pe_threads = 4 * a.rows;
-  const bool pe = gt < pe_threads;
-  const int64_t u = pe ? gt : gt - pe_threads;
-  const int64_t g = pe ? (u >> 2) : (u >> 6);
-  const int part = static_cast<int>(pe ? (u & 3) : (u & 63));
+__global__ void __launch_bounds__(kSplitThreadsPerRow * kSplitMaxRowsPerBlock) mla_epilogue_split_kernel(const Args a) {
+  const int lane = static_cast<int>(threadIdx.x) & 31;
+  const int warp = static_cast<int>(threadIdx.x) >> 5;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x / kSplitThreadsPerRow) + warp / 3;
+  const int part = warp % 3;
   if (g < a.rows) {
     if (g < a.T) {
-      small_cache_row<KVF8, ROPE>(a, g, pe, part);
+      split_cache_row<KVF8, ROPE>(a, g, part, lane);
     } else {
-      small_query_row<QF8, ROPE>(a, g - a.T, pe, part);
+      split_query_row<QF8, ROPE>(a, g - a.T, part, lane);
     }
   }
   pdl_trigger();
 }
 
-// kernel tables indexed by (ROPE, Q_FP8, KV_FP8) = flags & 7
+// kernel table indexed by (ROPE, Q_FP8, KV_FP8) = flags & 7
 template <int F>
-const void* small_kernel_for() {
+const void* split_kernel_for() {
   return reinterpret_cast<const void*>(
-      &mla_epilogue_small_kernel<(F & MLA_FLAG_Q_FP8) != 0, (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
+      &mla_epilogue_split_kernel<(F & MLA_FLAG_Q_FP8) != 0, (F & MLA_FLAG_KV_FP8) != 0, (F & MLA_FLAG_ROPE) != 0>);
 }
 
-const void* const kSplitKernels[8] = {small_kernel_for<0>(), small_kernel_for<1>(), small_kernel_for<2>(),
-                                      small_kernel_for<3>(), small_kernel_for<4>(), small_kernel_for<5>(),
-                                      small_kernel_for<6>(), small_kernel_for<7>()};
+const void* const kSplitKernels[8] = {split_kernel_for<0>(), split_kernel_for<1>(), split_kernel_for<2>(),
+                                      split_kernel_for<3>(), split_kernel_for<4>(), split_kernel_for<5>(),
+                                      split_kernel_for<6>(), split_kernel_for<7>()};
 
 // ------------------------------------------------------------------------------------
 // host helpers shared by every launcher (mla_runtime.h)
@@ -323,14 +197,12 @@ bool one_force_flag(uint32_t flags) {
   return !((flags & MLA_FLAG_FORCE_SPLIT) && (flags & MLA_FLAG_FORCE_ROWS));
 }
 
-// Threads per SPLIT block: the tuning value, or (0) the smallest multiple of
-// 32 that gives at most one block per SM, between 32 and 1024.
-int32_t split_threads(int64_t rows, int32_t sm_count) {
-  if (g_tuning.split_threads_per_block > 0) return g_tuning.split_threads_per_block;
-  const int64_t threads = mla::kSmallThreadsPerRow * rows;
-  int64_t per = (threads + sm_count - 1) / sm_count;
-  per = (per + 31) / 32 * 32;
-  return static_cast<int32_t>(per < 32 ? 32 : (per > mla::kSmallMaxThreads ? mla::kSmallMaxThreads : per));
+// Rows per SPLIT block: the tuning value, or (0) ceil(rows / SMs), so that
+// every SM gets a block before any block gets a second row.
+int32_t split_rows(int64_t rows, int32_t sm_count) {
+  if (g_tuning.split_rows_per_block > 0) return g_tuning.split_rows_per_block;
+  const int64_t r = (rows + sm_count - 1) / sm_count;
+  return static_cast<int32_t>(r < mla::kSplitMaxRowsPerBlock ? r : mla::kSplitMaxRowsPerBlock);
 }
 
 mla_status make_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla_plan* p) {
@@ -340,15 +212,11 @@ mla_status make_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla
                                                       : rows <= g_tuning.split_max_rows;
   p->sm_count = sm_count;
   if (split) {
-    const int32_t tpb = split_threads(rows, sm_count);
+    const int32_t rpb = split_rows(rows, sm_count);
     p->mode = MLA_MODE_SPLIT;
-    p->rows_per_block = 0;
-    p->threads_per_block = tpb;
-    p->blocks = (mla::kSmallThreadsPerRow * rows + tpb - 1) / tpb;
-    if (p->blocks > INT_MAX) {  // a small tuned block size on a huge forced launch
-      p->threads_per_block = mla::kSmallMaxThreads;
-      p->blocks = (mla::kSmallThreadsPerRow * rows + mla::kSmallMaxThreads - 1) / mla::kSmallMaxThreads;
-    }
+    p->rows_per_block = rpb;
+    p->threads_per_block = mla::kSplitThreadsPerRow * rpb;
+    p->blocks = (rows + rpb - 1) / rpb;
   } else {
     mla::rows_plan(rows, (flags & MLA_FLAG_Q_FP8) != 0, (flags & MLA_FLAG_KV_FP8) != 0, sm_count,
                    g_tuning.rows_blocks_per_sm, g_tuning.rows_warps_per_block, p);
@@ -376,11 +244,11 @@ int32_t mla_last_cuda_error(void) { return mla::g_last_cuda_error; }
 void mla_epilogue_set_tuning(const mla_tuning* t) {
   if (t == nullptr) return;
   if (t->split_max_rows > 0) g_tuning.split_max_rows = t->split_max_rows;
-  if (t->split_threads_per_block > 0) {
-    const int32_t v = (t->split_threads_per_block + 31) / 32 * 32;
-    g_tuning.split_threads_per_block = v < mla::kSmallMaxThreads ? v : mla::kSmallMaxThreads;
-  } else if (t->split_threads_per_block < 0) {
-    g_tuning.split_threads_per_block = 0;  // back to the automatic block size
+  if (t->split_rows_per_block > 0) {
+    g_tuning.split_rows_per_block =
+        t->split_rows_per_block < mla::kSplitMaxRowsPerBlock ? t->split_rows_per_block : mla::kSplitMaxRowsPerBlock;
+  } else if (t->split_rows_per_block < 0) {
+    g_tuning.split_rows_per_block = 0;  // back to the automatic choice
   }
   if (t->rows_warps_per_block > 0)
     g_tuning.rows_warps_per_block =
@@ -482,9 +350,6 @@ mla_status mla_epilogue_launch(
   a.q_out = static_cast<uint8_t*>(q_out);
   a.cache = static_cast<uint8_t*>(cache);
   a.status = status;
-  a.qpe_vec = aligned(q_pe, 16) && (T == 1 || q_pe_stride_t % 8 == 0) && (H == 1 || q_pe_stride_h % 8 == 0);
-  a.kpe_vec = aligned(k_pe, 16) && (T == 1 || k_pe_stride_t % 8 == 0);
-  a.tab_vec = rope && aligned(cos_sin, 16);
 
   const int k = static_cast<int>(flags & 7u);
   const void* fn = nullptr;

@@ -34,72 +34,6 @@ namespace rows {
 constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 6 : 5; }
 static_assert(rows_blocks_per_sm(true, true) <= kRowsMaxBlocksPerSm, "tuning limit covers the resident count");
 
-// Rotation of pair `i` for token t: (cos, sin) from the table row of its position.
-struct Rot {
-  float c, s;
-  bool on;
-};
-
-__device__ __forceinline__ Rot load_rotation(const Args& a, int64_t t, int i) {
-  Rot r{1.0f, 0.0f, false};
-  const int64_t pos = __ldg(a.positions + t);
-  if (pos >= 0 && pos < a.rope_rows) {
-    const float* row = a.cos_sin + pos * kPe;
-    r.c = __ldg(row + i);
-    r.s = __ldg(row + kHalfPe + i);
-    r.on = true;
-  }
-  return r;
-}
-
-template <bool FP8, bool FAST>
-__device__ __forceinline__ void store_nope(uint8_t* dst, int chunk, const uint4 v, const Divisor& d) {
-  if constexpr (FP8) {
-    *reinterpret_cast<uint2*>(dst + chunk * 8) = chunk_to_e4m3<FAST>(v, d);
-  } else {
-    *reinterpret_cast<uint4*>(dst + chunk * 16) = v;
-  }
-}
-
-// RoPE pair i of a row: pe[i] in the low half of `pe`, pe[i+32] in the high half.
-template <bool FP8, bool ROPE, bool FAST>
-__device__ __forceinline__ void store_pe(uint8_t* dst, int i, uint32_t pe, const Rot& r, const Divisor& d) {
-  float a = bf16_lo(pe);
-  float b = bf16_hi(pe);
-  bool rotated = false;
-  if constexpr (ROPE) {
-    if (r.on) {
-      float ya, yb;
-      rope_pair(a, b, r.c, r.s, ya, yb);
-      a = ya;
-      b = yb;
-      rotated = true;
-    }
-  }
-  if constexpr (FP8) {
-    const uint32_t p = e4m3x2_of_f32<FAST>(a, b, d);
-    dst[kNope + i] = static_cast<uint8_t>(p & 0xffu);
-    dst[kNope + kHalfPe + i] = static_cast<uint8_t>((p >> 8) & 0xffu);
-  } else {
-    const uint32_t p = rotated ? pack_bf16x2(a, b) : pe;  // unrotated: the input bits
-    uint16_t* o = reinterpret_cast<uint16_t*>(dst);
-    o[kNope + i] = static_cast<uint16_t>(p & 0xffffu);
-    o[kNope + kHalfPe + i] = static_cast<uint16_t>(p >> 16);
-  }
-}
-
-__device__ __forceinline__ uint4 ld_chunk(const uint16_t* row, int chunk) {
-  return __ldcg(reinterpret_cast<const uint4*>(row) + chunk);
-}
-
-__device__ __forceinline__ uint32_t ld_pair(const uint16_t* pe, int i) {
-  return static_cast<uint32_t>(__ldcg(pe + i)) | (static_cast<uint32_t>(__ldcg(pe + kHalfPe + i)) << 16);
-}
-
-// ------------------------------------------------------------------------------------
-// rows kernel: one warp per row, grid-stride over rows
-// ------------------------------------------------------------------------------------
-
 template <bool QF8, bool KVF8, bool ROPE, bool FAST>
 __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, const Divisor& dk) {
   const int lane = threadIdx.x & 31;

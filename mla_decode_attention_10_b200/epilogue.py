@@ -60,7 +60,7 @@ class mla_plan(ctypes.Structure):
 
 
 class mla_tuning(ctypes.Structure):
-    _fields_ = [("split_max_rows", ctypes.c_int64), ("split_threads_per_block", ctypes.c_int32),
+    _fields_ = [("split_max_rows", ctypes.c_int64), ("split_rows_per_block", ctypes.c_int32),
                 ("rows_warps_per_block", ctypes.c_int32), ("rows_blocks_per_sm", ctypes.c_int32)]
 
 
@@ -126,9 +126,9 @@ def mla_epilogue_plan(T: int, H: int, flags: int = 0, sm_count: int = 0) -> mla_
     return p
 
 
-def mla_epilogue_set_tuning(split_max_rows: int = 0, split_threads_per_block: int = 0,
+def mla_epilogue_set_tuning(split_max_rows: int = 0, split_rows_per_block: int = 0,
                             rows_warps_per_block: int = 0, rows_blocks_per_sm: int = 0) -> None:
-    t = mla_tuning(split_max_rows, split_threads_per_block, rows_warps_per_block, rows_blocks_per_sm)
+    t = mla_tuning(split_max_rows, split_rows_per_block, rows_warps_per_block, rows_blocks_per_sm)
     lib().mla_epilogue_set_tuning(ctypes.byref(t))
 
 

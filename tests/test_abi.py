@@ -135,11 +135,11 @@ def test_size_one_dimensions_skip_stride_checks(lib):
 
 def test_plan_modes_and_grids(lib):
     t = E.mla_epilogue_get_tuning()
-    assert t.split_threads_per_block == 0  # automatic block size
+    assert t.split_rows_per_block == 0  # automatic
     p = E.mla_epilogue_plan(64, 16, 0, sm_count=148)
-    assert p.mode == E.MLA_MODE_SPLIT and p.rows_per_block == 0
-    # 68 threads per row over about one block per SM: 64 * 17 * 68 / 148 -> 512
-    assert p.threads_per_block == 512 and p.blocks == -(-64 * 17 * 68 // 512) <= 148
+    # 64 * 17 = 1088 rows over 148 SMs: 8 rows (three warps each) per block
+    assert p.mode == E.MLA_MODE_SPLIT and p.rows_per_block == 8 and p.threads_per_block == 96 * 8
+    assert p.blocks == -(-64 * 17 // 8) <= 148
     # the default split threshold counts rows: 4608 = 271 tokens x 17 rows, rounded up
     assert t.split_max_rows == 4608
     assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
@@ -152,23 +152,21 @@ def test_plan_modes_and_grids(lib):
     assert p.blocks <= 148 * t.rows_blocks_per_sm
     assert E.mla_epilogue_plan(1, 16, E.MLA_FLAG_FORCE_ROWS, sm_count=148).mode == E.MLA_MODE_ROWS
     big = E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148)
-    assert big.mode == E.MLA_MODE_SPLIT and big.threads_per_block == 1024
-    assert big.blocks == -(-8192 * 17 * 68 // 1024)
+    assert big.mode == E.MLA_MODE_SPLIT and big.rows_per_block == 10 and big.blocks == -(-8192 * 17 // 10)
     with pytest.raises(E.MlaError):
         E.mla_epilogue_plan(0, 16, 0, sm_count=148)
     with pytest.raises(E.MlaError):
         E.mla_epilogue_plan(4, 16, E.MLA_FLAG_FORCE_SPLIT | E.MLA_FLAG_FORCE_ROWS, sm_count=148)
 
 
-@pytest.mark.parametrize("T,H,threads,blocks", [(1, 16, 32, 37), (1, 1, 32, 5), (1, 128, 64, 138), (4, 16, 32, 145),
-                                                (16, 16, 128, 145), (2, 16, 32, 73)])
-def test_decode_sizes_spread_over_the_sms(lib, T, H, threads, blocks):
-    """At decode sizes the plan gives about one block per SM, so a single
-    token's rows run on as many SMs as possible (one-warp blocks)."""
+@pytest.mark.parametrize("T,H,rpb,blocks", [(1, 16, 1, 17), (1, 1, 1, 2), (1, 128, 1, 129), (4, 16, 1, 68),
+                                            (16, 16, 2, 136), (2, 16, 1, 34), (32, 16, 4, 136)])
+def test_decode_sizes_spread_over_the_sms(lib, T, H, rpb, blocks):
+    """At decode sizes every SM gets a block before a block gets a second row:
+    a single token runs one row per SM (the num_tokens == 1 case)."""
     p = E.mla_epilogue_plan(T, H, E.MLA_FLAG_ROPE, sm_count=148)
     assert p.mode == E.MLA_MODE_SPLIT
-    assert (p.threads_per_block, p.blocks) == (threads, blocks)
-    assert p.blocks * p.threads_per_block >= T * (H + 1) * 68
+    assert (p.rows_per_block, p.threads_per_block, p.blocks) == (rpb, 96 * rpb, blocks)
 
 
 def test_tuning_moves_the_threshold_and_clamps(lib):
@@ -177,20 +175,20 @@ def test_tuning_moves_the_threshold_and_clamps(lib):
         E.mla_epilogue_set_tuning(split_max_rows=64 * 17)
         assert E.mla_epilogue_plan(64, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
         assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_ROWS
-        E.mla_epilogue_set_tuning(split_threads_per_block=5000, rows_warps_per_block=99, rows_blocks_per_sm=99)
+        E.mla_epilogue_set_tuning(split_rows_per_block=99, rows_warps_per_block=99, rows_blocks_per_sm=99)
         t = E.mla_epilogue_get_tuning()
-        assert t.split_threads_per_block == 1024
+        assert t.split_rows_per_block == 10
         assert t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 6
-        E.mla_epilogue_set_tuning(split_threads_per_block=200)  # rounded up to whole warps
+        E.mla_epilogue_set_tuning(split_rows_per_block=3)
         p = E.mla_epilogue_plan(5, 16, 0, sm_count=148)
-        assert p.threads_per_block == 224 and p.blocks == -(-5 * 17 * 68 // 224)
+        assert p.rows_per_block == 3 and p.threads_per_block == 288 and p.blocks == 29
         E.mla_epilogue_set_tuning()  # all zero: unchanged
         assert E.mla_epilogue_get_tuning().split_max_rows == 64 * 17
-        assert E.mla_epilogue_get_tuning().split_threads_per_block == 224
-        E.mla_epilogue_set_tuning(split_threads_per_block=-1)  # back to automatic
-        assert E.mla_epilogue_get_tuning().split_threads_per_block == 0
+        assert E.mla_epilogue_get_tuning().split_rows_per_block == 3
+        E.mla_epilogue_set_tuning(split_rows_per_block=-1)  # back to automatic
+        assert E.mla_epilogue_get_tuning().split_rows_per_block == 0
     finally:
-        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_threads_per_block or -1,
+        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_rows_per_block or -1,
                                   old.rows_warps_per_block, old.rows_blocks_per_sm)
 
 

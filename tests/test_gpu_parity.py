@@ -66,11 +66,11 @@ def test_flag_combinations_and_shapes(flags, T, H):
 @pytest.mark.parametrize("flags", list(range(8)))
 @pytest.mark.parametrize("H", [1, 16, 27, 28, 128])
 def test_single_token_behind_producer(flags, H):
-    """T = 1 through the plan's own choice (one-warp blocks spread over the
-    SMs, rows straddling blocks), launched with PDL behind the synthetic
-    producer, every flag combination."""
+    """T = 1 through the plan's own choice (one row per block, spread over
+    the SMs), launched with PDL behind the synthetic producer, every flag
+    combination."""
     p = E.mla_epilogue_plan(1, H, flags)
-    assert p.mode == E.MLA_MODE_SPLIT and p.threads_per_block <= 64
+    assert p.mode == E.MLA_MODE_SPLIT and p.rows_per_block == 1
     w = W.make("token", 1, H, flags, seed=600 + H * 8 + flags, num_blocks=2, std=2.0, rope_rows=1024,
                scale=0.05, cache_fill="random")
     check_workload(w, producer=True)
@@ -115,24 +115,23 @@ def test_rows_kernel_warp_counts(warps):
         check_workload(w, extra_flags=E.MLA_FLAG_FORCE_ROWS)
         check_workload(w, extra_flags=E.MLA_FLAG_FORCE_ROWS, producer=True)
     finally:
-        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_threads_per_block or -1, old.rows_warps_per_block,
+        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_rows_per_block or -1, old.rows_warps_per_block,
                                   old.rows_blocks_per_sm)
 
 
-@pytest.mark.parametrize("threads", [32, 96, 544, 1024])
-def test_split_kernel_block_sizes(threads):
-    """Any whole-warp block size: rows straddle blocks, nope and pe threads of
-    one row sit in different blocks."""
+@pytest.mark.parametrize("rpb", [1, 3, 10])
+def test_split_kernel_rows_per_block(rpb):
+    """Blocks of 1 .. 10 rows, the last one ragged."""
     old = E.mla_epilogue_get_tuning()
     try:
-        E.mla_epilogue_set_tuning(split_threads_per_block=threads)
-        w = W.make("tpb", 37, 7, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8, seed=threads, num_blocks=8, std=2.0,
+        E.mla_epilogue_set_tuning(split_rows_per_block=rpb)
+        w = W.make("rpb", 37, 7, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8, seed=rpb, num_blocks=8, std=2.0,
                    rope_rows=512, scale=0.05, cache_fill="random")
-        assert E.mla_epilogue_plan(37, 7, E.MLA_FLAG_FORCE_SPLIT).threads_per_block == threads
+        assert E.mla_epilogue_plan(37, 7, E.MLA_FLAG_FORCE_SPLIT).rows_per_block == rpb
         check_workload(w, extra_flags=E.MLA_FLAG_FORCE_SPLIT)
         check_workload(w, extra_flags=E.MLA_FLAG_FORCE_SPLIT, producer=True)
     finally:
-        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_threads_per_block or -1, old.rows_warps_per_block,
+        E.mla_epilogue_set_tuning(old.split_max_rows, old.split_rows_per_block or -1, old.rows_warps_per_block,
                                   old.rows_blocks_per_sm)
 
 
