@@ -75,8 +75,8 @@ typedef enum mla_status {
 
 /* Kernel choice (mla_plan.mode). */
 #define MLA_MODE_SPLIT 1 /* small T: three warps per 576-wide row (two move 16-byte nope chunks, one rotates the
-                            32 RoPE pairs, one per lane); rows_per_block rows per block, ceil(rows / SMs) unless
-                            tuned, so a single token's rows run one per SM */
+                            32 RoPE pairs, one per lane); rows_per_block rows per block, ceil(rows / SMs) up to 4
+                            unless tuned, so a single token's rows run one per SM */
 #define MLA_MODE_ROWS  2 /* large T: one warp per row, grid-stride, grid sized to the resident blocks */
 
 /*
@@ -177,8 +177,8 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  * default threshold counts rows, not tokens.
  *   split_max_rows       T * (H + 1) at or below which MLA_MODE_SPLIT is used (default 4608)
  *   split_rows_per_block rows per block in MLA_MODE_SPLIT (block = 96 * this), at most
- *                        10; 0 (default) takes ceil(rows / SMs); a negative value
- *                        restores the default
+ *                        10; 0 (default) takes ceil(rows / SMs), at most 4; a negative
+ *                        value restores the default
  *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8 (default 8)
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
  *                        the number the kernel's register cap keeps resident (6 with

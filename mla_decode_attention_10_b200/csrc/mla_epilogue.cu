@@ -16,9 +16,9 @@
 //     (i, i+32), one pair per lane, so the rotation needs no shuffles and
 //     each thread's chain of dependent work stays short.  A block holds R
 //     rows; at decode sizes latency falls as the rows spread over more SMs
-//     (measured on B200), so the plan takes R = ceil(rows / SMs): one row per
-//     block for a single token (the num_tokens == 1 case of PR #53526,
-//     关联脉络), more rows per block only once every SM has one.
+//     (measured on B200), so the plan takes R = ceil(rows / SMs), at most 4:
+//     one row per block for a single token (the num_tokens == 1 case of
+//     PR #53526, 关联脉络), more rows per block only once every SM has one.
 //   ROWS (large T): mla_rows.cu.
 //
 // In SPLIT every thread computes its addresses and loads its slot,
@@ -42,6 +42,7 @@ namespace mla {
 
 constexpr int kSplitThreadsPerRow = 96;  // three warps
 constexpr int kSplitMaxRowsPerBlock = 10;  // 960 threads
+constexpr int kSplitAutoMaxRows = 4;       // the automatic choice stops at 4 rows (measured best at T = 64 .. 256)
 
 // A row's e4m3 scale: its load is issued with the row's other loads and the
 // divisor is made only when the stores need it, so the scale adds no step
@@ -197,12 +198,12 @@ bool one_force_flag(uint32_t flags) {
   return !((flags & MLA_FLAG_FORCE_SPLIT) && (flags & MLA_FLAG_FORCE_ROWS));
 }
 
-// Rows per SPLIT block: the tuning value, or (0) ceil(rows / SMs), so that
-// every SM gets a block before any block gets a second row.
+// Rows per SPLIT block: the tuning value, or (0) ceil(rows / SMs) up to 4,
+// so that every SM gets a block before any block gets a second row.
 int32_t split_rows(int64_t rows, int32_t sm_count) {
   if (g_tuning.split_rows_per_block > 0) return g_tuning.split_rows_per_block;
   const int64_t r = (rows + sm_count - 1) / sm_count;
-  return static_cast<int32_t>(r < mla::kSplitMaxRowsPerBlock ? r : mla::kSplitMaxRowsPerBlock);
+  return static_cast<int32_t>(r < mla::kSplitAutoMaxRows ? r : mla::kSplitAutoMaxRows);
 }
 
 mla_status make_plan(int64_t T, int64_t H, uint32_t flags, int32_t sm_count, mla_plan* p) {

@@ -137,9 +137,9 @@ def test_plan_modes_and_grids(lib):
     t = E.mla_epilogue_get_tuning()
     assert t.split_rows_per_block == 0  # automatic
     p = E.mla_epilogue_plan(64, 16, 0, sm_count=148)
-    # 64 * 17 = 1088 rows over 148 SMs: 8 rows (three warps each) per block
-    assert p.mode == E.MLA_MODE_SPLIT and p.rows_per_block == 8 and p.threads_per_block == 96 * 8
-    assert p.blocks == -(-64 * 17 // 8) <= 148
+    # 64 * 17 = 1088 rows over 148 SMs: 8 rows a block would do, the automatic choice stops at 4
+    assert p.mode == E.MLA_MODE_SPLIT and p.rows_per_block == 4 and p.threads_per_block == 96 * 4
+    assert p.blocks == 64 * 17 // 4
     # the default split threshold counts rows: 4608 = 271 tokens x 17 rows, rounded up
     assert t.split_max_rows == 4608
     assert E.mla_epilogue_plan(65, 16, 0, sm_count=148).mode == E.MLA_MODE_SPLIT
@@ -152,7 +152,7 @@ def test_plan_modes_and_grids(lib):
     assert p.blocks <= 148 * t.rows_blocks_per_sm
     assert E.mla_epilogue_plan(1, 16, E.MLA_FLAG_FORCE_ROWS, sm_count=148).mode == E.MLA_MODE_ROWS
     big = E.mla_epilogue_plan(8192, 16, E.MLA_FLAG_FORCE_SPLIT, sm_count=148)
-    assert big.mode == E.MLA_MODE_SPLIT and big.rows_per_block == 10 and big.blocks == -(-8192 * 17 // 10)
+    assert big.mode == E.MLA_MODE_SPLIT and big.rows_per_block == 4 and big.blocks == 8192 * 17 // 4
     with pytest.raises(E.MlaError):
         E.mla_epilogue_plan(0, 16, 0, sm_count=148)
     with pytest.raises(E.MlaError):
@@ -160,7 +160,7 @@ def test_plan_modes_and_grids(lib):
 
 
 @pytest.mark.parametrize("T,H,rpb,blocks", [(1, 16, 1, 17), (1, 1, 1, 2), (1, 128, 1, 129), (4, 16, 1, 68),
-                                            (16, 16, 2, 136), (2, 16, 1, 34), (32, 16, 4, 136)])
+                                            (16, 16, 2, 136), (2, 16, 1, 34), (32, 16, 4, 136), (64, 16, 4, 272)])
 def test_decode_sizes_spread_over_the_sms(lib, T, H, rpb, blocks):
     """At decode sizes every SM gets a block before a block gets a second row:
     a single token runs one row per SM (the num_tokens == 1 case)."""
