@@ -1,7 +1,7 @@
 """Benchmark of the fused MLA decode epilogue on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-sweep] [--no-cpu-baseline]
+                    [--workload NAME] [--no-sweep] [--no-cpu-baseline] [--split-policy]
 
 One step is one call of the epilogue (the whole hot path) on one batch of
 the workload.  Default workload: the large batch, T=8192 tokens, H=16 heads,
@@ -66,8 +66,12 @@ KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
                   "mla_decode_attention_10_b200/csrc/mla_rows.cu",
                   "mla_decode_attention_10_b200/csrc/epilogue_device.cuh",
                   "mla_decode_attention_10_b200/csrc/latent_math.cuh", "include/mla_epilogue.h")
-TRAFFIC_SOURCE_HASH = None
-TRAFFIC_BYTES = {}
+TRAFFIC_SOURCE_HASH = "070e905add0f644a"
+TRAFFIC_BYTES = {
+    "batch_t8192_h16_pdl_fp8": 163992832 + 53276672,
+    "split_boundary_t64_h16_rope": 1278208 + 0,
+    "prefill_t1024_h128_strided": 152627456 + 102022400,
+}
 L2_BYTES = 126 * 2 ** 20
 GRAPH_CALLS = 500
 # ---------------------------------------------------------------------------------------
@@ -567,6 +571,49 @@ def producer_consumer_chain(hx, ds, device, calls, reps):
     return out
 
 
+def split_policy(args):
+    """The split / rows crossover: both kernels forced on the same cold
+    inputs (RoPE, Q and KV e4m3, std 2, random-byte cache) across T for
+    H in {8, 16, 32, 128}; one JSON line per (T, H)."""
+    from mla_decode_attention_10_b200 import epilogue as E
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    peak, _ = measured_hbm_gbs()
+
+    def forced(force):
+        class Forced(Harness):
+            def epilogue(self, ds, extra=0):
+                return Harness.epilogue(self, ds, extra | force)
+
+            def empty(self, w0, flags):
+                plan = E.mla_epilogue_plan(w0.T, w0.H, w0.flags | force)
+
+                def f(i):
+                    rc = E.mla_harness_empty(plan.blocks, plan.threads_per_block, flags, stream.cuda_stream)
+                    if rc != E.MLA_OK:
+                        raise E.MlaError(rc, "mla_harness_empty")
+                return f, plan
+        return Forced(E, stream)
+
+    grid = {8: (128, 256, 384, 512, 768), 16: (128, 192, 256, 384, 512), 32: (64, 96, 128, 192, 256),
+            128: (16, 24, 32, 48, 64)}
+    for H, Ts in grid.items():
+        for T in Ts:
+            name = f"split_policy_t{T}_h{H}"
+            W.RECIPES[name] = dict(T=T, H=H, flags=W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8, seed=0,
+                                   num_blocks=max(64, 4 * T), std=2.0, rope_rows=32768, scale=0.05,
+                                   cache_fill="random", recipe=f"T={T} H={H}, RoPE, Q/KV e4m3, std 2")
+            ds = DeviceSets(name)
+            row = {"T": T, "H": H, "rows": T * (H + 1)}
+            for mode, force in (("split", E.MLA_FLAG_FORCE_SPLIT), ("rows", E.MLA_FLAG_FORCE_ROWS)):
+                row[mode + "_us"] = standalone(forced(force), ds, device, 200, 7, peak)["us_per_call"]
+            row["plan"] = "split" if E.mla_epilogue_plan(T, H, 0).mode == E.MLA_MODE_SPLIT else "rows"
+            print(json.dumps(row), flush=True)
+            del ds
+            torch.cuda.empty_cache()
+
+
 def common_config(name: str):
     """The `config` both arms print (plus their own `implementation`)."""
     w = W.RECIPES[name]
@@ -985,6 +1032,8 @@ def parse(argv=None):
     p.add_argument("--workload", default=HEADLINE, choices=W.names())
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--split-policy", action="store_true",
+                   help="measure the split / rows crossover instead (one JSON line per shape)")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be at least 3")
@@ -996,6 +1045,9 @@ def parse(argv=None):
 def main(argv=None):
     args = parse(argv)
     rank, world, local_rank = rank_info()
+    if args.split_policy:
+        split_policy(args)
+        return 0
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
