@@ -67,3 +67,24 @@ def test_bench_rejects_short_warmup():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"],
                        capture_output=True, text=True, timeout=120)
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_reference_arm_samples_token_slices_of_the_workload():
+    """With a small time budget the reference arm runs the oracle on a token
+    slice of the workload and scales its time to a full call; the slice is
+    the workload's first tokens with the same cache, table and scales."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from mla_decode_attention_10_b200 import workloads as W
+    w = W.named("decode_sweep_t64_h16_rope_fp8")
+    s = bench.token_slice(w, 5)
+    assert s.T == 5 and s.H == w.H and s.q_nope.shape[0] == 5 and s.slot_mapping.shape[0] == 5
+    assert s.positions.shape[0] == 5 and s.cache is w.cache and s.cos_sin is w.cos_sin
+    assert bench.token_slice(w, 64) is w
+    args = bench.parse(["--impl", "reference", "--steps", "2", "--warmup", "3",
+                        "--workload", "decode_sweep_t64_h16_rope_fp8"])
+    line = bench.run_reference(args, 0, 1, budget_s=1e-6)   # forces the smallest slice
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert "of the 64 tokens" in line["cpu_baseline"]["sample"] and "scaled by 64/" in line["cpu_baseline"]["sample"]
+    assert line["config"] == dict(bench.common_config("decode_sweep_t64_h16_rope_fp8"),
+                                  implementation=line["config"]["implementation"])
