@@ -19,7 +19,7 @@
 //   * same report, key-source listing of test_decode_epilogue_row_split_boundary:
 //     q == cat(ql_nope, q_pe) and cache rows at slot_mapping == cat(kv_c, k_pe)
 //     when neither RoPE nor FP8 is on.
-// Readings where the pages are silent (each also listed in the design doc):
+// Readings where the pages are silent:
 //   * RoPE is rotate-half over the pairs (i, i+32) of the 64 pe dims, with a
 //     fp32 table row [cos_0..cos_31 | sin_0..sin_31] per position; one position
 //     per token, shared by all of its rows.  Computed in fp32, no contraction.
