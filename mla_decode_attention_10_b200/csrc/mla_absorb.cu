@@ -55,7 +55,7 @@ constexpr int kPe = 64;
 constexpr int kHalfPe = 32;
 constexpr int kRow = 576;
 constexpr int kTmaWarp = 0, kMmaWarp = 1, kEpiWarp0 = 2, kEpiWarps = 8, kPeWarp0 = 10, kPeWarps = 6;
-constexpr int kThreads = 32 * (kPeWarp0 + kPeWarps);  // 448
+constexpr int kThreads = 32 * (kPeWarp0 + kPeWarps);  // 512: the register file at 128 a thread
 constexpr int kStages = 2;                            // A ring
 constexpr uint32_t kSlabA = kM * 64 * 2;     // one 64-wide column slab of A: 16 KB
 constexpr uint32_t kSlabB = kN * 64 * 2;     // one 64-wide column slab of B: 32 KB
