@@ -65,6 +65,20 @@ MLA_API mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t c
                                  unsigned long long* result, mla_stream_t stream);
 
 /*
+ * Device check of the e4m3 bytes of bf16 inputs over many scales: for every
+ * scale bit pattern in [first, first + count) and every one of the 65536
+ * bf16 values x, compares the e4m3 byte the epilogue stores for x / scale
+ * with the byte of CUDA's IEEE quotient __fdiv_rn.  (The epilogue reaches
+ * bf16 quotients in one corrected step; they may differ from the IEEE
+ * quotient in the last bit but not in the e4m3 byte.)  result (device,
+ * 2 x uint64, 8-byte aligned, overwritten): [0] differing (scale, x) pairs,
+ * [1] smallest scale pattern with one (UINT64_MAX if none).
+ * first + count <= 2^32.  Work: count x 65536 quotients per call.
+ */
+MLA_API mla_status mla_harness_bf16_scale_check(uint32_t first, uint32_t count, unsigned long long* result,
+                                                mla_stream_t stream);
+
+/*
  * Synthetic downstream consumer standing in for the attention kernel that
  * reads the epilogue's outputs (PR #54896 report, 实现拆解 item 2: the
  * epilogue's trigger lets the attention kernel overlap with it).  For every

@@ -140,13 +140,44 @@ __device__ __forceinline__ uint32_t e4m3x2_of_f32(float lo, float hi, const Divi
   return pack_e4m3x2(qlo, qhi);
 }
 
+// One corrected step of the quotient above: q0 = RN(x y), q1 = RN(q0 + r y).
+// q1 may differ from the IEEE quotient in its last bit, but when x is a bf16
+// value (8 significant bits) it has the same e4m3 byte.  Let z = x / s.
+// q0 + r y = z + (z - q0)(s y - 1) with |s y - 1| <= 2^-24 and
+// |z - q0| < 2 ulp(z), so it lies within 2^-23 ulp(z) of z.  Two adjacent
+// fp32 values round to different e4m3 bytes only when one of them is an
+// e4m3 rounding midpoint M (odd significand M' of at most 5 bits), so the
+// bytes of q1 and RN(z) can differ only if z lies that close to a point
+// m = M +- (half the fp32 spacing on that side of M).  In units of
+// ulp(s) ulp(z) / 2, s m is the integer S (M' 2^k +- 1), with S the 24-bit
+// significand of s and 20 <= k <= 25, and x would lie within 4 units of it.
+// Modulo 2^k that forces S = c 2^k + r with |r| < 4, and then
+// S (M' 2^k +- 1) = c M' 2^2k + (+-c + r M') 2^k +- r spans more than 8
+// significant bits unless +-c + r M' = 0.  The only such case is
+// M = 2^-10, S = 2^24 - 1 (s just below a power of two), where evaluating
+// the two steps exactly gives q1 = RN(z).
+__device__ __forceinline__ void quotient_pair_neg1(float mlo, float mhi, const Divisor& d, float& qlo,
+                                                   float& qhi) {
+  asm("{\n\t"
+      ".reg .b64 mx, q, r;\n\t"
+      "mov.b64 mx, {%2, %3};\n\t"
+      "mul.rn.f32x2 q, mx, %5;\n\t"
+      "fma.rn.f32x2 r, q, %4, mx;\n\t"
+      "fma.rn.f32x2 q, r, %5, q;\n\t"
+      "mov.b64 {%0, %1}, q;\n\t"
+      "}"
+      : "=f"(qlo), "=f"(qhi)
+      : "f"(mlo), "f"(mhi), "l"(d.s2), "l"(d.ny2));
+}
+
 // e4m3 bytes of the two bf16 of `w` divided by s (low half in bits 0..7).
+// FAST takes the one-step quotient (exact in e4m3 for bf16 inputs, above).
 template <bool FAST>
 __device__ __forceinline__ uint32_t e4m3x2_of_bf16x2(uint32_t w, const Divisor& d) {
   float qlo, qhi;
   if (FAST) {
     const uint32_t m = neg_clamp_bf16x2(w, d);
-    quotient_pair_neg(bf16_lo(m), bf16_hi(m), d, qlo, qhi);
+    quotient_pair_neg1(bf16_lo(m), bf16_hi(m), d, qlo, qhi);
   } else {
     qlo = __fdiv_rn(bf16_lo(w), d.s);
     qhi = __fdiv_rn(bf16_hi(w), d.s);

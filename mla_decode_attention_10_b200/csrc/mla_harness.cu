@@ -88,6 +88,38 @@ __global__ void __launch_bounds__(256) div_check_kernel(float scale, uint64_t fi
   if (lowest != ~0ull) atomicMin(result + 2, lowest);
 }
 
+// Every bf16 value through the epilogue's e4m3 path against the byte of the
+// IEEE quotient, for scale bit patterns [first, first + count).  Item i is
+// scale first + i / 8 and bf16 pairs (2k, 2k + 1) for k in one eighth of
+// [0, 32768).
+__global__ void __launch_bounds__(256) bf16_scale_check_kernel(uint32_t first, uint32_t count,
+                                                               unsigned long long* result) {
+  constexpr uint32_t kParts = 8, kPairs = 32768 / kParts;
+  const uint64_t items = static_cast<uint64_t>(count) * kParts;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  unsigned long long bad = 0, lowest = ~0ull;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < items; i += stride) {
+    const uint32_t bits = first + static_cast<uint32_t>(i / kParts);
+    const float scale = __uint_as_float(bits);
+    const Divisor d = make_divisor(scale);
+    const uint32_t k0 = static_cast<uint32_t>(i % kParts) * kPairs;
+    uint32_t n = 0;
+    for (uint32_t k = k0; k < k0 + kPairs; ++k) {
+      const uint32_t w = ((2u * k + 1u) << 16) | (2u * k);
+      const uint32_t got = d.fast ? e4m3x2_of_bf16x2<true>(w, d) : e4m3x2_of_bf16x2<false>(w, d);
+      const uint32_t ref = pack_e4m3x2(__fdiv_rn(bf16_lo(w), scale), __fdiv_rn(bf16_hi(w), scale));
+      n += ((got ^ ref) & 0xffu) != 0u;
+      n += ((got ^ ref) & 0xff00u) != 0u;
+    }
+    if (n != 0u) {
+      bad += n;
+      if (bits < lowest) lowest = bits;
+    }
+  }
+  if (bad) atomicAdd(result + 0, bad);
+  if (lowest != ~0ull) atomicMin(result + 1, lowest);
+}
+
 // e4m3 byte -> fp32 (exact: every e4m3 value is an fp16 value).
 __device__ __forceinline__ float e4m3_to_f32(uint8_t b) {
   uint32_t h2;
@@ -204,6 +236,24 @@ mla_status mla_harness_div_check(float scale, uint64_t first, uint64_t count, un
   void* args[] = {&scale, &first, &count, &result};
   return launch(reinterpret_cast<const void*>(&div_check_kernel), dim3(static_cast<unsigned>(sms) * 16), dim3(256),
                 false, s, args);
+}
+
+mla_status mla_harness_bf16_scale_check(uint32_t first, uint32_t count, unsigned long long* result,
+                                        mla_stream_t stream) {
+  using namespace mla::harness;
+  if (result == nullptr || (reinterpret_cast<uintptr_t>(result) & 7u) != 0) return MLA_ERR_INVALID_ARG;
+  if (static_cast<uint64_t>(first) + count > (UINT64_C(1) << 32)) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(result, 0, sizeof(unsigned long long), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(result + 1, 0xff, sizeof(unsigned long long), s);
+  if (e != cudaSuccess) return finish(e);
+  if (count == 0) return MLA_OK;
+  int32_t sms = 0;
+  const mla_status st = mla::current_device(nullptr, &sms);
+  if (st != MLA_OK) return st;
+  void* args[] = {&first, &count, &result};
+  return launch(reinterpret_cast<const void*>(&bf16_scale_check_kernel), dim3(static_cast<unsigned>(sms) * 16),
+                dim3(256), false, s, args);
 }
 
 mla_status mla_harness_consume(const void* q_out, const void* cache, const int64_t* slot_mapping, int64_t T,

@@ -101,6 +101,8 @@ def lib() -> ctypes.CDLL:
                                         vp, vp, vp]
         L.mla_harness_div_check.restype = ctypes.c_int
         L.mla_harness_div_check.argtypes = [ctypes.c_float, u64, u64, vp, vp]
+        L.mla_harness_bf16_scale_check.restype = ctypes.c_int
+        L.mla_harness_bf16_scale_check.argtypes = [u32, u32, vp, vp]
         _lib = L
     return _lib
 
@@ -162,6 +164,10 @@ def mla_harness_consume(q_out, cache, slot_mapping, T, H, cache_rows, flags, sco
 
 def mla_harness_div_check(scale: float, first: int, count: int, result, stream) -> int:
     return lib().mla_harness_div_check(scale, first, count, result, stream)
+
+
+def mla_harness_bf16_scale_check(first: int, count: int, result, stream) -> int:
+    return lib().mla_harness_bf16_scale_check(first, count, result, stream)
 
 
 def mla_absorb_launch(q_nope_c, q_nope_c_stride_t, q_nope_c_stride_h, w_uk, q_pe, q_pe_stride_t, q_pe_stride_h,

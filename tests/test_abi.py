@@ -214,6 +214,9 @@ def test_harness_validation(lib, kw, code):
     assert E.mla_harness_empty(1, 2048, 0, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_div_check(1.0, 0, 2 ** 32 + 1, A, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_div_check(1.0, 0, 1, None, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_bf16_scale_check(2 ** 32 - 4, 5, A, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_bf16_scale_check(0, 1, None, None) == E.MLA_ERR_INVALID_ARG
+    assert E.mla_harness_bf16_scale_check(0, 1, A + 4, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_consume(A, A, A, 4, 16, 64, 64, A, None) == E.MLA_ERR_UNSUPPORTED
     assert E.mla_harness_consume(A, A, A, -1, 16, 64, 0, A, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_consume(None, A, A, 4, 16, 64, 0, A, None) == E.MLA_ERR_INVALID_ARG

@@ -194,6 +194,27 @@ def test_quotient_equals_ieee_division_for_every_fp32(scale):
     assert (bad_q, bad_b) == (0, 0), f"scale {scale}: {bad_q} quotients, {bad_b} bytes differ, first 0x{first & 0xffffffff:08x}"
 
 
+# every scale significand of a binade: 2^23 scales x 65536 bf16 values each;
+# the edges of the fast range, the bench's 0.05 (binade -5) and a few others
+BF16_SCALE_BINADES = [-64, -9, -5, 0, 10, 63]
+
+
+@pytest.mark.parametrize("e", BF16_SCALE_BINADES)
+def test_bf16_bytes_equal_ieee_division_for_every_scale_of_a_binade(e):
+    """The e4m3 byte of every bf16 value divided by every fp32 scale in
+    [2^e, 2^(e+1)) equals the byte of CUDA's IEEE quotient (the epilogue's
+    bf16 quotient takes one corrected step, exact in e4m3 but not in fp32)."""
+    first = (e + 127) << 23
+    res = torch.zeros(2, dtype=torch.int64, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    chunk = 1 << 21
+    for c in range((1 << 23) // chunk):
+        rc = E.mla_harness_bf16_scale_check(first + c * chunk, chunk, res.data_ptr(), stream)
+        assert rc == E.MLA_OK
+        bad, lowest = res.cpu().tolist()
+        assert bad == 0, f"{bad} bytes differ, first at scale 0x{lowest & 0xffffffff:08x}"
+
+
 # ---- edge cases
 
 def test_zero_tokens_touches_nothing():
