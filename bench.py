@@ -66,11 +66,9 @@ KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
                   "mla_decode_attention_10_b200/csrc/mla_rows.cu",
                   "mla_decode_attention_10_b200/csrc/epilogue_device.cuh",
                   "mla_decode_attention_10_b200/csrc/latent_math.cuh", "include/mla_epilogue.h")
-TRAFFIC_SOURCE_HASH = "070e905add0f644a"
+TRAFFIC_SOURCE_HASH = "344ebd9364cf6c2b"
 TRAFFIC_BYTES = {
-    "batch_t8192_h16_pdl_fp8": 163992832 + 53276672,
-    "split_boundary_t64_h16_rope": 1278208 + 0,
-    "prefill_t1024_h128_strided": 152627456 + 102022400,
+    "batch_t8192_h16_pdl_fp8": 163928832 + 50717952,
 }
 L2_BYTES = 126 * 2 ** 20
 GRAPH_CALLS = 500
@@ -699,7 +697,7 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": round(us, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": config,
         "timing": {"mode": mode_name(E, plan), "grid": [plan.blocks, plan.threads_per_block],
                    "regions": REPLAYS, "region_us_per_call_sorted": spread,
@@ -1013,7 +1011,7 @@ def run_reference(args, rank, world, budget_s: float = 150.0):
     cb = {"value": round(us, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
     return {"impl": "reference", "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 4),
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": dict(common_config(args.workload), implementation="CPU oracle (oracle/mla_oracle.cpp), "
                                                                         "one host thread"),

@@ -77,7 +77,8 @@ typedef enum mla_status {
 #define MLA_MODE_SPLIT 1 /* small T: three warps per 576-wide row (two move 16-byte nope chunks, one rotates the
                             32 RoPE pairs, one per lane); rows_per_block rows per block, ceil(rows / SMs) up to 4
                             unless tuned, so a single token's rows run one per SM */
-#define MLA_MODE_ROWS  2 /* large T: one warp per row, grid-stride, grid sized to the resident blocks */
+#define MLA_MODE_ROWS  2 /* large T: grid-stride over rows, grid sized to the resident blocks; one warp per row
+                            (bf16 outputs) or half a warp per row (an e4m3 output) */
 
 /*
  * mla_epilogue_launch -- the whole epilogue in one kernel launch.
@@ -160,8 +161,8 @@ typedef struct mla_plan {
   int32_t mode;              /* MLA_MODE_SPLIT or MLA_MODE_ROWS */
   int32_t threads_per_block;
   int64_t blocks;
-  int32_t rows_per_block;    /* SPLIT: rows one block covers (96 threads each); ROWS: 1 (one row per warp at a
-                                time) */
+  int32_t rows_per_block;    /* SPLIT: rows one block covers (96 threads each); ROWS: rows one warp converts at
+                                a time (1, or 2 with an e4m3 output) */
   int32_t sm_count;
 } mla_plan;
 
@@ -181,7 +182,7 @@ MLA_API mla_status mla_epilogue_plan(int64_t T, int64_t H, uint32_t flags, int32
  *                        value restores the default
  *   rows_warps_per_block warps per block in MLA_MODE_ROWS, at most 8 (default 8)
  *   rows_blocks_per_sm   blocks per SM the MLA_MODE_ROWS grid is sized for, at most
- *                        the number the kernel's register cap keeps resident (6 with
+ *                        the number the kernel's register cap keeps resident (4 with
  *                        an e4m3 output, 5 without; default: that number)
  * Larger values are clamped to those limits; 0 keeps the current setting.
  */

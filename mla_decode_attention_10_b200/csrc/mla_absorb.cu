@@ -303,7 +303,9 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
         : "r"(bar), "r"(parity)
         : "memory");
     if (done) return true;
-    if (*abort_flag != 0u) return false;
+    // the flag is read every 16 tries: shared-memory reads beside the tensor
+    // cores' and the copy engine's traffic each cost about ten wavefronts
+    if ((i & 15u) == 15u && *abort_flag != 0u) return false;
   }
   return false;
 }
@@ -469,7 +471,13 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
     for (int i = 0; i < count; ++i) {
       const TileCoord c = tile_at(first + i, mt);
       const int b = i & 1;
-      const bool ready = wait_or_abort(smem_u32(&bars.acc_full[b]), static_cast<uint32_t>(i / 2) & 1u, abort_flag);
+      // lane 0 polls for its warp; the barrier below orders the other lanes
+      // after its wait, and the tcgen05 fence after the barrier orders the
+      // accumulator reads after it
+      bool ready = true;
+      if (lane == 0)
+        ready = wait_or_abort(smem_u32(&bars.acc_full[b]), static_cast<uint32_t>(i / 2) & 1u, abort_flag) &&
+                *abort_flag == 0u;
       // e4m3 tiles (32 KB) alternate between the two halves of the 64 KB
       // staging area: wait only for the stores of two tiles back, which read
       // the half this tile writes; bf16 tiles fill it and wait for the last
@@ -480,7 +488,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
           asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
       }
-      if (!bar_and(1, 32 * kEpiWarps, ready && *abort_flag == 0u)) {
+      if (!bar_and(1, 32 * kEpiWarps, ready)) {
         if (lane == 0 && ew == 0) {
           *abort_flag = 1u;
           report(p.status, MLA_STATUS_TIMEOUT);

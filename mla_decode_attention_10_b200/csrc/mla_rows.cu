@@ -1,14 +1,17 @@
 // mla_rows.cu -- the large-batch (MLA_MODE_ROWS) kernel of the fused MLA
-// decode epilogue: one warp per row, grid-stride over rows, the grid sized to
-// the resident blocks on every SM.
+// decode epilogue: a fixed group of lanes per row, grid-stride over rows, the
+// grid sized to the resident blocks on every SM.
 //
 // The rows of a call are the cache rows [0, T), then the query rows in q_out
-// order (vLLM PR #54896 report, 实现拆解 items 1-3).  Warp w of the grid
-// takes rows w, w + W, w + 2W, ... (W = all warps of the grid), so all warps
-// walk one window of memory together.  Lane l moves nope chunks l and l + 32
-// (16 bytes each) and rotates pe pair (l, l + 32): the e4m3 arithmetic of a
-// row is spread over all 32 lanes, which matters because the e4m3 kernel is
-// bound by instruction issue as much as by memory (measured on B200).
+// order (vLLM PR #54896 report, 实现拆解 items 1-3).  A warp converts 32 / L
+// adjacent rows per trip (L lanes each) and then moves on by the number of
+// warps in the grid, so all warps walk one window of memory together.  Lane l
+// of a row moves nope chunks l + k L (16 bytes each) and rotates the pe pairs
+// (i, i + 32) for i = l + k L.  With an e4m3 output L = 16: the kernel is
+// bound by instruction issue (measured on B200), and two rows per warp trip
+// halve the per-row instructions (addresses, slot, position, table row,
+// checks) while the e4m3 arithmetic stays spread over all 32 lanes.  bf16
+// outputs, bound by memory, keep L = 32 (one row per warp).
 //
 // Query rows execute griddepcontrol.wait once, before their first read of
 // q_nope / q_pe (the upstream kernel writes them); cache rows, slots,
@@ -28,12 +31,13 @@
 namespace mla {
 namespace rows {
 
-// Resident 256-thread blocks per SM the kernel is compiled for: 5 (a
-// 48-register cap) for bf16 outputs; 6 (40 registers) when an output is
-// e4m3, whose arithmetic leaves the kernel short of memory parallelism at 5
-// (measured on B200: 0.75 -> 0.78 of copy bandwidth for T=8192, H=16; the
-// bf16 variants lose at 6).
-constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 6 : 5; }
+// Lanes per row and resident 256-thread blocks per SM the kernel is compiled
+// for.  e4m3 outputs: 16 lanes per row at 4 blocks (64 registers; measured on
+// B200 at T=8192, H=16: 40.1 us against 42.5 for one warp per row at 6
+// blocks and 41.0 at 5).  bf16 outputs: one warp per row at 5 blocks (48
+// registers; 49.9 us at T=1024, H=128 against 53.4 for 16 lanes per row).
+__host__ __device__ constexpr int rows_lanes_per_row(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 16 : 32; }
+constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 4 : 5; }
 static_assert(rows_blocks_per_sm(true, true) <= kRowsMaxBlocksPerSm, "tuning limit covers the resident count");
 
 // q / H for the row loop.  64-bit rows: one multiply-high by ceil(2^64 / H)
@@ -63,13 +67,15 @@ __device__ __forceinline__ uint32_t div_h(const HeadDiv32& d, const Args&, uint3
 __device__ __forceinline__ int64_t div_h(const HeadDiv32&, const Args& a, int64_t q) { return div_heads(a, q); }
 
 // Idx: the integer type of the row loop.  e4m3 outputs use 32 bits, unsigned
-// so that g + warps (rows < 2^31 plus the grid's warps) cannot wrap: the
-// e4m3 kernel is bound by instruction issue, and 32-bit indexing saves a
+// so that the trip counter times rows per trip cannot wrap (rows < 2^31):
+// the e4m3 kernel is bound by instruction issue, and 32-bit indexing saves a
 // tenth of its instructions (measured on B200: 47.2 -> 44.2 us at T=8192,
 // H=16); bf16 outputs, bound by memory, keep 64 bits (2% faster there).
-template <typename Idx, bool QF8, bool KVF8, bool ROPE, bool FAST>
+template <int L, typename Idx, bool QF8, bool KVF8, bool ROPE, bool FAST>
 __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, const Divisor& dk) {
-  const int lane = threadIdx.x & 31;
+  constexpr int kRowsPerTrip = 32 / L, kChunks = 64 / L, kPairs = 32 / L;
+  const int ll = threadIdx.x & (L - 1);
+  const Idx sub = static_cast<Idx>((threadIdx.x & 31) / L);
   const HeadDiv32 hd = head_div32(a.H);
   const Idx H = static_cast<Idx>(a.H);
   const Idx T = static_cast<Idx>(a.T);
@@ -79,7 +85,9 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
   const Idx wid = static_cast<Idx>(blockIdx.x) * static_cast<Idx>(blockDim.x >> 5) + static_cast<Idx>(threadIdx.x >> 5);
   bool waited = false;
 
-  for (Idx g = wid; g < rows; g += warps) {
+  for (Idx trip = wid; trip * kRowsPerTrip < rows; trip += warps) {
+    const Idx g = trip * kRowsPerTrip + sub;
+    if (g >= rows) continue;
     // 1. addresses, slot and rotation: nothing here depends on the upstream kernel
     const bool is_cache = g < T;
     Idx t;
@@ -93,7 +101,7 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
       const int64_t slot = __ldg(a.slots + t);
       if (slot >= 0 && slot < a.cache_rows) {
         dst = a.cache + slot * (KVF8 ? kRow : 2 * kRow);
-      } else if (slot >= a.cache_rows && lane == 0) {
+      } else if (slot >= a.cache_rows && ll == 0) {
         report(a.status, MLA_STATUS_SLOT_RANGE);
       }
     } else {
@@ -104,16 +112,21 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
       pe = a.q_pe + static_cast<int64_t>(t) * a.qp_st + static_cast<int64_t>(h) * a.qp_sh;
       dst = a.q_out + static_cast<int64_t>(q) * (QF8 ? kRow : 2 * kRow);
     }
-    Rot rot{1.0f, 0.0f, false};
+    Rot rot[kPairs];
+#pragma unroll
+    for (int k = 0; k < kPairs; ++k) rot[k] = Rot{1.0f, 0.0f, false};
     if constexpr (ROPE) {
       const int32_t pos = __ldg(a.positions + t);
       if (pos >= 0 && pos < rope_rows) {
         const float* row = a.cos_sin + static_cast<int64_t>(pos) * kPe;
-        rot.c = __ldg(row + lane);
-        rot.s = __ldg(row + kHalfPe + lane);
-        rot.on = true;
+#pragma unroll
+        for (int k = 0; k < kPairs; ++k) {
+          rot[k].c = __ldg(row + ll + k * L);
+          rot[k].s = __ldg(row + kHalfPe + ll + k * L);
+          rot[k].on = true;
+        }
       }
-      if (is_cache && lane == 0 && !rot.on) report(a.status, MLA_STATUS_POS_RANGE);
+      if (is_cache && ll == 0 && !rot[0].on) report(a.status, MLA_STATUS_POS_RANGE);
     }
 
     // 2. query rows read what the upstream kernel wrote: wait for it once
@@ -123,18 +136,23 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
     }
 
     // 3. the row's loads, then 4. convert and store
-    const uint4 n0 = ld_chunk(nope, lane);
-    const uint4 n1 = ld_chunk(nope, lane + 32);
-    const uint32_t p = ld_pair(pe, lane);
+    uint4 n[kChunks];
+    uint32_t p[kPairs];
+#pragma unroll
+    for (int k = 0; k < kChunks; ++k) n[k] = ld_chunk(nope, ll + k * L);
+#pragma unroll
+    for (int k = 0; k < kPairs; ++k) p[k] = ld_pair(pe, ll + k * L);
     if (dst == nullptr) continue;
     if (is_cache) {
-      store_nope<KVF8, FAST>(dst, lane, n0, dk);
-      store_nope<KVF8, FAST>(dst, lane + 32, n1, dk);
-      store_pe<KVF8, ROPE, FAST>(dst, lane, p, rot, dk);
+#pragma unroll
+      for (int k = 0; k < kChunks; ++k) store_nope<KVF8, FAST>(dst, ll + k * L, n[k], dk);
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) store_pe<KVF8, ROPE, FAST>(dst, ll + k * L, p[k], rot[k], dk);
     } else {
-      store_nope<QF8, FAST>(dst, lane, n0, dq);
-      store_nope<QF8, FAST>(dst, lane + 32, n1, dq);
-      store_pe<QF8, ROPE, FAST>(dst, lane, p, rot, dq);
+#pragma unroll
+      for (int k = 0; k < kChunks; ++k) store_nope<QF8, FAST>(dst, ll + k * L, n[k], dq);
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) store_pe<QF8, ROPE, FAST>(dst, ll + k * L, p[k], rot[k], dq);
     }
   }
 }
@@ -148,10 +166,11 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps, rows_blocks_per_sm(QF8, KV
   if constexpr (QF8) dq = make_divisor(__ldg(a.q_scale));
   if constexpr (KVF8) dk = make_divisor(__ldg(a.kv_scale));
   using Idx = std::conditional_t<QF8 || KVF8, uint32_t, int64_t>;
+  constexpr int L = rows_lanes_per_row(QF8, KVF8);
   if (dq.fast && dk.fast) {
-    rows_body<Idx, QF8, KVF8, ROPE, true>(a, dq, dk);
+    rows_body<L, Idx, QF8, KVF8, ROPE, true>(a, dq, dk);
   } else {
-    rows_body<Idx, QF8, KVF8, ROPE, false>(a, dq, dk);
+    rows_body<L, Idx, QF8, KVF8, ROPE, false>(a, dq, dk);
   }
   pdl_trigger();
 }
@@ -170,12 +189,13 @@ const void* const kKernels[8] = {kernel_for<0>(), kernel_for<1>(), kernel_for<2>
 void rows_plan(int64_t rows, bool qf8, bool kvf8, int32_t sm_count, int32_t blocks_per_sm, int32_t warps_per_block,
                mla_plan* p) {
   const int32_t w = warps_per_block < kRowsMaxWarps ? warps_per_block : kRowsMaxWarps;
-  const int64_t need = (rows + w - 1) / w;
+  const int64_t per_block = static_cast<int64_t>(w) * (32 / rows::rows_lanes_per_row(qf8, kvf8));
+  const int64_t need = (rows + per_block - 1) / per_block;
   const int32_t resident = rows::rows_blocks_per_sm(qf8, kvf8);
   const int32_t per_sm = blocks_per_sm < resident ? blocks_per_sm : resident;
   const int64_t cap = static_cast<int64_t>(sm_count) * per_sm;
   p->mode = MLA_MODE_ROWS;
-  p->rows_per_block = 1;
+  p->rows_per_block = 32 / rows::rows_lanes_per_row(qf8, kvf8);
   p->threads_per_block = 32 * w;
   p->blocks = need < cap ? need : cap;
 }

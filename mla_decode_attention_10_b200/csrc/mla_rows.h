@@ -11,7 +11,7 @@ namespace mla {
 
 // Upper limits (and defaults) of the tuning knobs mla_epilogue_set_tuning
 // clamps to.
-constexpr int kRowsMaxBlocksPerSm = 6;  // resident blocks per SM the kernel is compiled for
+constexpr int kRowsMaxBlocksPerSm = 5;  // resident blocks per SM the kernels are compiled for, at most
 constexpr int kRowsMaxWarps = 8;        // warps per block
 constexpr int kRowsDefaultWarps = 8;
 

@@ -178,7 +178,7 @@ def test_tuning_moves_the_threshold_and_clamps(lib):
         E.mla_epilogue_set_tuning(split_rows_per_block=99, rows_warps_per_block=99, rows_blocks_per_sm=99)
         t = E.mla_epilogue_get_tuning()
         assert t.split_rows_per_block == 10
-        assert t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 6
+        assert t.rows_warps_per_block == 8 and t.rows_blocks_per_sm == 5
         E.mla_epilogue_set_tuning(split_rows_per_block=3)
         p = E.mla_epilogue_plan(5, 16, 0, sm_count=148)
         assert p.rows_per_block == 3 and p.threads_per_block == 288 and p.blocks == 29
