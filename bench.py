@@ -69,8 +69,14 @@ KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
 TRAFFIC_SOURCE_HASH = "344ebd9364cf6c2b"
 TRAFFIC_BYTES = {
     "batch_t8192_h16_pdl_fp8": 163928832 + 50717952,
+    "split_boundary_t64_h16_rope": 1279488 + 0,
+    "prefill_t1024_h128_strided": 152629760 + 101840128,
 }
 L2_BYTES = 126 * 2 ** 20
+# The weight-streaming producer (decode sizes): the weights a projection
+# producing q for 16 heads reads, and the pool its calls rotate over.
+GEMM_WEIGHT_BYTES = 9 * 2 ** 20
+GEMM_WEIGHT_POOL_BYTES = 32 * GEMM_WEIGHT_BYTES
 GRAPH_CALLS = 500
 # ---------------------------------------------------------------------------------------
 # ranks
@@ -395,6 +401,27 @@ class Harness:
                 raise E.MlaError(rc, "mla_harness_produce")
         return f
 
+    def producer_after_weights(self, ds, pool, sink):
+        """The producer that first streams GEMM_WEIGHT_BYTES of weights: call i
+        reads window i of `pool` (more than 2x L2 in all), so its weights come
+        from DRAM as a projection's would between layers."""
+        E, stream, S = self.E, self.stream, len(ds.sets)
+        windows = pool.numel() * pool.element_size() // GEMM_WEIGHT_BYTES
+
+        def f(i):
+            d, _, src = ds.sets[i % S]
+            if src is None:
+                nxt = ds.sets[(i + 1) % S][0]
+                src = (nxt.q_nope, nxt.q_pe)
+            wptr = pool.data_ptr() + (i % windows) * GEMM_WEIGHT_BYTES
+            rc = E.mla_harness_produce_after_weights(
+                src[0].data_ptr(), src[1].data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0), d.q_nope.stride(1),
+                d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1), wptr, GEMM_WEIGHT_BYTES, sink.data_ptr(),
+                d.T, d.H, 0, stream.cuda_stream)
+            if rc != E.MLA_OK:
+                raise E.MlaError(rc, "mla_harness_produce_after_weights")
+        return f
+
     def runner(self, step, calls, warmup=3):
         warm = GraphRunner(step, max(warmup, 1), self.stream)
         warm.replay()
@@ -413,15 +440,16 @@ def then(*fns):
     return f
 
 
-def behind_producer(hx, ds, device, calls, reps):
+def behind_producer(hx, ds, device, calls, reps, prod=None, prefix=""):
     """Per call: the synthetic producer writes the query inputs, then X is
     launched as its programmatic dependent (PDL).  X is the epilogue, the
     empty kernel (same grid) and the empty kernel that executes
     griddepcontrol.wait; each increment is X's cost over the producer alone.
     The floor of a dependent launch is the empty kernel that waits: one that
-    does not wait runs beside the producer and is not a dependent at all."""
+    does not wait runs beside the producer and is not a dependent at all.
+    `prod` replaces the plain producer (keys then start with `prefix`)."""
     E = hx.E
-    prod = hx.producer(ds)
+    prod = prod or hx.producer(ds)
     empty, _ = hx.empty(ds.w0, E.MLA_FLAG_PDL)
     empty_wait, _ = hx.empty(ds.w0, E.MLA_FLAG_PDL | E.MLA_HARNESS_EMPTY_WAIT)
     steps = {"producer_us": prod,
@@ -443,7 +471,7 @@ def behind_producer(hx, ds, device, calls, reps):
     out["empty_wait_increment_us"] = round(inc_wait, 4)
     out["empty_increment_us"] = round(inc_empty, 4)
     out["floor_ratio_behind_producer"] = round(inc / inc_wait, 3) if inc_wait > 0 else None
-    return out
+    return {prefix + k: v for k, v in out.items()}
 
 
 def standalone(hx, ds, device, calls, reps, peak):
@@ -475,20 +503,28 @@ def mode_name(E, plan):
 def decode_floors(hx, device, peak, calls=200, reps=7):
     """T = 1 .. 64 (the decode sweep workload: H=16, RoPE, e4m3): standalone
     with cold inputs (`floor_ratio`: against an empty kernel of the same
-    grid), and behind the producer with PDL: `floor_ratio_behind_producer`
+    grid), and behind two producers with PDL: the plain one, which only
+    copies q, and `gemm_`, which first streams GEMM_WEIGHT_BYTES of weights
+    as the projection that produces q would.  `floor_ratio_behind_producer`
     is the epilogue's increment over the producer against the increment of
     an empty dependent that waits, `increment_over_launch_floor` the same
     increment against one bare launch of an empty kernel."""
     out = []
+    pool = torch.ones(GEMM_WEIGHT_POOL_BYTES // 4, dtype=torch.int32, device=device)
+    sink = torch.zeros(1, dtype=torch.int32, device=device)
     for T in DECODE_T:
         ds = DeviceSets(f"decode_sweep_t{T}_h16_rope_fp8")
         row = standalone(hx, ds, device, calls, reps, peak)
         row.update(behind_producer(hx, ds, device, calls, reps))
-        # the epilogue's cost behind the producer against one bare launch
+        row.update(behind_producer(hx, ds, device, calls, reps, hx.producer_after_weights(ds, pool, sink), "gemm_"))
+        # the epilogue's cost behind each producer against one bare launch
         row["increment_over_launch_floor"] = round(row["epilogue_increment_pdl_us"] / row["launch_floor_us"], 3)
+        row["gemm_increment_over_launch_floor"] = round(row["gemm_epilogue_increment_pdl_us"] /
+                                                        row["launch_floor_us"], 3)
         out.append(row)
         del ds
         torch.cuda.empty_cache()
+    del pool, sink
     return out
 
 

@@ -38,6 +38,24 @@ MLA_API mla_status mla_harness_produce(const void* src_nope, const void* src_pe,
                                int64_t T, int64_t H, uint32_t flags, mla_stream_t stream);
 
 /*
+ * The same producer with the duration of a real one: before it writes q it
+ * reads `weight_bytes` of `weights` through all of its blocks, as the
+ * projection GEMM streams its weight matrix before its epilogue writes the
+ * query (PR #54896 report, 实现拆解 item 2: the epilogue's loads that do not
+ * depend on the GEMM overlap the GEMM's tail).  Every block XORs the 32-bit
+ * words it read into *sink (device, 4-byte aligned), so after one call *sink
+ * is its old value XOR every word of the weights.  The grid covers all SMs
+ * (4 blocks of 256 threads each) however small T is.  weights: 16-byte
+ * aligned, weight_bytes a multiple of 16 (0 reads nothing).  Otherwise as
+ * mla_harness_produce.
+ */
+MLA_API mla_status mla_harness_produce_after_weights(const void* src_nope, const void* src_pe,
+                               void* q_nope, int64_t q_nope_stride_t, int64_t q_nope_stride_h,
+                               void* q_pe, int64_t q_pe_stride_t, int64_t q_pe_stride_h,
+                               const void* weights, int64_t weight_bytes, uint32_t* sink,
+                               int64_t T, int64_t H, uint32_t flags, mla_stream_t stream);
+
+/*
  * An empty kernel launched with `blocks` x `threads` and, with MLA_FLAG_PDL,
  * the programmatic-serialization attribute: the bare-launch floor that the
  * epilogue's latency at decode sizes is compared with.  With

@@ -14,13 +14,26 @@ namespace harness {
 
 // One warp per (token, head) row: 1024 bytes of nope (two 16-byte chunks per
 // lane) and 128 bytes of pe (lanes 0..7), grid-stride.
+// With `weights`: first every thread reads its grid-stride share of the
+// weights (16-byte words) and each block XORs what it read into *sink.
 __global__ void __launch_bounds__(256) produce_kernel(const uint4* __restrict__ src_nope,
                                                       const uint4* __restrict__ src_pe,
                                                       uint16_t* q_nope, int64_t qn_st, int64_t qn_sh,
                                                       uint16_t* q_pe, int64_t qp_st, int64_t qp_sh,
-                                                      int64_t T, int64_t H) {
+                                                      int64_t T, int64_t H, const uint4* __restrict__ weights,
+                                                      int64_t weight_words, uint32_t* sink) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (weight_words > 0) {
+    const int64_t threads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    uint32_t acc = 0;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < weight_words; i += threads) {
+      const uint4 w = __ldcs(weights + i);
+      acc ^= w.x ^ w.y ^ w.z ^ w.w;
+    }
+    for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0 && acc != 0u) atomicXor(sink, acc);
+  }
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t rows = T * H;
@@ -176,37 +189,64 @@ mla_status launch(const void* fn, dim3 grid, dim3 block, bool pdl, cudaStream_t 
   return finish(cudaLaunchKernelExC(&cfg, fn, args));
 }
 
-}  // namespace harness
-}  // namespace mla
-
-extern "C" {
-
-mla_status mla_harness_produce(const void* src_nope, const void* src_pe, void* q_nope, int64_t q_nope_stride_t,
-                               int64_t q_nope_stride_h, void* q_pe, int64_t q_pe_stride_t, int64_t q_pe_stride_h,
-                               int64_t T, int64_t H, uint32_t flags, mla_stream_t stream) {
-  using namespace mla::harness;
+mla_status produce(const void* src_nope, const void* src_pe, void* q_nope, int64_t q_nope_stride_t,
+                   int64_t q_nope_stride_h, void* q_pe, int64_t q_pe_stride_t, int64_t q_pe_stride_h,
+                   const void* weights, int64_t weight_bytes, uint32_t* sink, int64_t T, int64_t H, uint32_t flags,
+                   mla_stream_t stream) {
   if ((flags & ~MLA_FLAG_PDL) != 0) return MLA_ERR_UNSUPPORTED;
-  if (T < 0 || H < 1 || T > (INT64_C(1) << 31) / H) return MLA_ERR_INVALID_ARG;
-  if (T == 0) return MLA_OK;
-  if (!src_nope || !src_pe || !q_nope || !q_pe) return MLA_ERR_INVALID_ARG;
-  if (q_nope_stride_t < 0 || q_nope_stride_h < 0 || q_pe_stride_t < 0 || q_pe_stride_h < 0)
-    return MLA_ERR_INVALID_ARG;
-  if (!aligned16(src_nope) || !aligned16(src_pe) || !aligned16(q_nope) || !aligned16(q_pe) ||
-      (q_nope_stride_t % 8) || (q_nope_stride_h % 8) || (q_pe_stride_t % 8) || (q_pe_stride_h % 8))
+  if (T < 0 || H < 1 || T > (INT64_C(1) << 31) / H || weight_bytes < 0) return MLA_ERR_INVALID_ARG;
+  if (weight_bytes > 0 && (weights == nullptr || sink == nullptr)) return MLA_ERR_INVALID_ARG;
+  if (weight_bytes > 0 && (!aligned16(weights) || (weight_bytes % 16) != 0 ||
+                           (reinterpret_cast<uintptr_t>(sink) & 3u) != 0))
     return MLA_ERR_ALIGNMENT;
+  if (T == 0 && weight_bytes == 0) return MLA_OK;
+  if (T > 0) {
+    if (!src_nope || !src_pe || !q_nope || !q_pe) return MLA_ERR_INVALID_ARG;
+    if (q_nope_stride_t < 0 || q_nope_stride_h < 0 || q_pe_stride_t < 0 || q_pe_stride_h < 0)
+      return MLA_ERR_INVALID_ARG;
+    if (!aligned16(src_nope) || !aligned16(src_pe) || !aligned16(q_nope) || !aligned16(q_pe) ||
+        (q_nope_stride_t % 8) || (q_nope_stride_h % 8) || (q_pe_stride_t % 8) || (q_pe_stride_h % 8))
+      return MLA_ERR_ALIGNMENT;
+  }
   int32_t sms = 0;
   const mla_status s = mla::current_device(nullptr, &sms);
   if (s != MLA_OK) return s;
   const int64_t rows = T * H;
   int64_t blocks = (rows + 7) / 8;
   if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  if (weight_bytes > 0 && blocks < static_cast<int64_t>(sms) * 4) blocks = static_cast<int64_t>(sms) * 4;
   const uint4* sn = static_cast<const uint4*>(src_nope);
   const uint4* sp = static_cast<const uint4*>(src_pe);
   uint16_t* qn = static_cast<uint16_t*>(q_nope);
   uint16_t* qp = static_cast<uint16_t*>(q_pe);
-  void* args[] = {&sn, &sp, &qn, &q_nope_stride_t, &q_nope_stride_h, &qp, &q_pe_stride_t, &q_pe_stride_h, &T, &H};
+  const uint4* wt = static_cast<const uint4*>(weights);
+  int64_t words = weight_bytes / 16;
+  void* args[] = {&sn, &sp, &qn, &q_nope_stride_t, &q_nope_stride_h, &qp, &q_pe_stride_t, &q_pe_stride_h,
+                  &T, &H, &wt, &words, &sink};
   return launch(reinterpret_cast<const void*>(&produce_kernel), dim3(static_cast<unsigned>(blocks)), dim3(256),
                 (flags & MLA_FLAG_PDL) != 0, reinterpret_cast<cudaStream_t>(stream), args);
+}
+
+}  // namespace harness
+}  // namespace mla
+
+extern "C" {
+
+
+mla_status mla_harness_produce(const void* src_nope, const void* src_pe, void* q_nope, int64_t q_nope_stride_t,
+                               int64_t q_nope_stride_h, void* q_pe, int64_t q_pe_stride_t, int64_t q_pe_stride_h,
+                               int64_t T, int64_t H, uint32_t flags, mla_stream_t stream) {
+  return mla::harness::produce(src_nope, src_pe, q_nope, q_nope_stride_t, q_nope_stride_h, q_pe, q_pe_stride_t,
+                               q_pe_stride_h, nullptr, 0, nullptr, T, H, flags, stream);
+}
+
+mla_status mla_harness_produce_after_weights(const void* src_nope, const void* src_pe, void* q_nope,
+                                             int64_t q_nope_stride_t, int64_t q_nope_stride_h, void* q_pe,
+                                             int64_t q_pe_stride_t, int64_t q_pe_stride_h, const void* weights,
+                                             int64_t weight_bytes, uint32_t* sink, int64_t T, int64_t H,
+                                             uint32_t flags, mla_stream_t stream) {
+  return mla::harness::produce(src_nope, src_pe, q_nope, q_nope_stride_t, q_nope_stride_h, q_pe, q_pe_stride_t,
+                               q_pe_stride_h, weights, weight_bytes, sink, T, H, flags, stream);
 }
 
 mla_status mla_harness_empty(int64_t blocks, int32_t threads, uint32_t flags, mla_stream_t stream) {

@@ -92,6 +92,9 @@ def lib() -> ctypes.CDLL:
         L.mla_last_cuda_error.argtypes = []
         L.mla_harness_produce.restype = ctypes.c_int
         L.mla_harness_produce.argtypes = [vp, vp, vp, i64, i64, vp, i64, i64, i64, i64, u32, vp]
+        L.mla_harness_produce_after_weights.restype = ctypes.c_int
+        L.mla_harness_produce_after_weights.argtypes = [vp, vp, vp, i64, i64, vp, i64, i64, vp, i64, vp, i64, i64,
+                                                        u32, vp]
         L.mla_harness_empty.restype = ctypes.c_int
         L.mla_harness_empty.argtypes = [i64, i32, u32, vp]
         L.mla_harness_consume.restype = ctypes.c_int
@@ -152,6 +155,14 @@ def mla_harness_produce(src_nope, src_pe, q_nope, q_nope_stride_t, q_nope_stride
                         q_pe_stride_t, q_pe_stride_h, T, H, flags, stream) -> int:
     return lib().mla_harness_produce(src_nope, src_pe, q_nope, q_nope_stride_t, q_nope_stride_h,
                                      q_pe, q_pe_stride_t, q_pe_stride_h, T, H, flags, stream)
+
+
+def mla_harness_produce_after_weights(src_nope, src_pe, q_nope, q_nope_stride_t, q_nope_stride_h, q_pe,
+                                     q_pe_stride_t, q_pe_stride_h, weights, weight_bytes, sink, T, H, flags,
+                                     stream) -> int:
+    return lib().mla_harness_produce_after_weights(src_nope, src_pe, q_nope, q_nope_stride_t, q_nope_stride_h, q_pe,
+                                                   q_pe_stride_t, q_pe_stride_h, weights, weight_bytes, sink, T, H,
+                                                   flags, stream)
 
 
 def mla_harness_empty(blocks: int, threads: int, flags: int, stream) -> int:

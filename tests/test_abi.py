@@ -215,6 +215,14 @@ def test_harness_validation(lib, kw, code):
     assert E.mla_harness_div_check(1.0, 0, 2 ** 32 + 1, A, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_div_check(1.0, 0, 1, None, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_bf16_scale_check(2 ** 32 - 4, 5, A, None) == E.MLA_ERR_INVALID_ARG
+    pw = dict(src_nope=A, src_pe=A, q_nope=A, q_nope_stride_t=16 * 512, q_nope_stride_h=512, q_pe=A,
+              q_pe_stride_t=16 * 64, q_pe_stride_h=64, weights=A, weight_bytes=1 << 20, sink=A, T=4, H=16, flags=0,
+              stream=None)
+    for kw, want in ((dict(weights=None), E.MLA_ERR_INVALID_ARG), (dict(sink=None), E.MLA_ERR_INVALID_ARG),
+                     (dict(weight_bytes=-16), E.MLA_ERR_INVALID_ARG), (dict(weight_bytes=24), E.MLA_ERR_ALIGNMENT),
+                     (dict(weights=A + 8), E.MLA_ERR_ALIGNMENT), (dict(sink=A + 2), E.MLA_ERR_ALIGNMENT),
+                     (dict(flags=4), E.MLA_ERR_UNSUPPORTED), (dict(T=0, weight_bytes=0), E.MLA_OK)):
+        assert E.mla_harness_produce_after_weights(**{**pw, **kw}) == want, kw
     assert E.mla_harness_bf16_scale_check(0, 1, None, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_bf16_scale_check(0, 1, A + 4, None) == E.MLA_ERR_INVALID_ARG
     assert E.mla_harness_consume(A, A, A, 4, 16, 64, 64, A, None) == E.MLA_ERR_UNSUPPORTED
@@ -266,6 +274,8 @@ def test_cuda_failures_are_recorded_for_every_launcher(lib):
         "mla_epilogue_plan": lambda: E.lib().mla_epilogue_plan(4, 16, 0, 0, ctypes.byref(E.mla_plan())),
         "mla_harness_produce": lambda: E.mla_harness_produce(A, A, A, 16 * 512, 512, A, 16 * 64, 64, 4, 16, 0, None),
         "mla_harness_empty": lambda: E.mla_harness_empty(1, 32, 0, None),
+        "mla_harness_produce_after_weights": lambda: E.mla_harness_produce_after_weights(
+            A, A, A, 16 * 512, 512, A, 16 * 64, 64, A, 1 << 20, A, 4, 16, 0, None),
         "mla_harness_consume": lambda: E.mla_harness_consume(A, A, A, 4, 16, 64, 0, A, None),
     }
     for name, call in calls.items():

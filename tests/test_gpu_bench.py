@@ -43,3 +43,21 @@ def test_bench_prints_one_contract_line():
     assert d["launch_floor_us"] > 0
     bp = d["behind_producer"]
     assert bp["producer_us"] > 0 and bp["epilogue_increment_pdl_us"] > 0
+
+
+def test_decode_floor_readings_behind_both_producers(monkeypatch):
+    """bench's decode readings at T=1, short: standalone, behind the plain
+    producer and behind the producer that streams weights first."""
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench as B
+    from mla_decode_attention_10_b200 import epilogue as E
+    monkeypatch.setattr(B, "DECODE_T", (1,))
+    dev = torch.device("cuda", 0)
+    hx = B.Harness(E, torch.cuda.Stream(dev))
+    (row,) = B.decode_floors(hx, dev, 6650.0, calls=20, reps=2)
+    assert row["T"] == 1 and row["mode"] == "split"
+    assert row["gemm_producer_us"] > row["producer_us"] > 0
+    for p in ("", "gemm_"):
+        assert row[p + "epilogue_increment_pdl_us"] > 0 and row[p + "empty_wait_increment_us"] > -1.0
+        assert row[p + "increment_over_launch_floor"] > 0

@@ -9,6 +9,7 @@ rows, computed in double precision on the host; q_out and the cache are
 checked bit for bit as well.
 """
 
+import numpy as np
 import pytest
 import torch
 
@@ -78,3 +79,35 @@ def test_consumer_marks_out_of_range_slots_nan():
     s = scores.view(5, 4)
     assert torch.isnan(s[2]).all() and torch.isnan(s[4]).all()
     assert not torch.isnan(s[[0, 1, 3]]).any()
+
+
+@pytest.mark.parametrize("T,flags", [(1, W.FLAG_ROPE | W.FLAG_Q_FP8 | W.FLAG_KV_FP8), (64, W.FLAG_ROPE)])
+def test_epilogue_behind_a_producer_that_streams_weights_first(T, flags):
+    """The producer reads 9 MiB of weights before it writes q (a projection
+    GEMM's duration); the epilogue runs as its programmatic dependent.  The
+    outputs are the oracle's bit for bit, and the producer's checksum of the
+    weights is the XOR of all their 32-bit words."""
+    w = W.make("gemm_like", T, 16, flags, seed=41 + T, num_blocks=8, rope_rows=4096, scale=0.05,
+               cache_fill="random")
+    d = w.to("cuda")
+    s = torch.cuda.current_stream()
+    g = torch.Generator().manual_seed(5)
+    weights_host = torch.randint(-2 ** 31, 2 ** 31 - 1, ((9 << 20) // 4,), dtype=torch.int32, generator=g)
+    weights = weights_host.to("cuda")
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    src_n, src_p = d.q_nope.contiguous().clone(), d.q_pe.contiguous().clone()
+    d.q_nope.fill_(float("nan"))
+    d.q_pe.fill_(float("nan"))
+    q_out = torch.empty((w.T, w.H, W.ROW), dtype=w.q_out_dtype(), device="cuda")
+    torch.cuda.synchronize()
+    assert E.mla_harness_produce_after_weights(
+        src_n.data_ptr(), src_p.data_ptr(), d.q_nope.data_ptr(), d.q_nope.stride(0), d.q_nope.stride(1),
+        d.q_pe.data_ptr(), d.q_pe.stride(0), d.q_pe.stride(1), weights.data_ptr(), weights.numel() * 4,
+        sink.data_ptr(), w.T, w.H, 0, s.cuda_stream) == E.MLA_OK
+    assert E.launch_workload(d, q_out, extra_flags=E.MLA_FLAG_PDL) == E.MLA_OK
+    torch.cuda.synchronize()
+    qo, co, _ = run_oracle(w)
+    assert_same(q_out.cpu(), qo, "q_out")
+    assert_same(d.cache.cpu(), co, "cache")
+    x = weights_host.numpy().view("uint32")
+    assert int(sink.cpu().numpy().view("uint32")[0]) == int(np.bitwise_xor.reduce(x))
