@@ -38,7 +38,9 @@ struct Args {
   const float* kv_scale;
   int64_t T;
   int64_t H;
-  uint64_t h_magic;  // ceil(2^64 / H) for H >= 2, see div_heads
+  uint64_t h_magic;   // ceil(2^64 / H) for H >= 2, see div_heads
+  uint32_t h_magic32;  // ceil(2^(31+s) / H), 2^(s-1) < H <= 2^s, for H >= 2; 0 for H = 1
+  uint32_t h_shift32;  // s - 1
   int64_t cache_rows;
   int64_t rows;  // T * (H + 1)
   uint8_t* q_out;

@@ -346,6 +346,14 @@ mla_status mla_epilogue_launch(
   a.T = T;
   a.H = H;
   a.h_magic = H > 1 ? (UINT64_MAX / static_cast<uint64_t>(H)) + 1 : 0;
+  {
+    uint32_t sh = 0;  // ceil(log2 H)
+    while ((INT64_C(1) << sh) < H) ++sh;
+    a.h_magic32 = H > 1 ? static_cast<uint32_t>(((UINT64_C(1) << (31 + sh)) + static_cast<uint64_t>(H) - 1) /
+                                                static_cast<uint64_t>(H))
+                        : 0u;
+    a.h_shift32 = H > 1 ? sh - 1 : 0u;
+  }
   a.cache_rows = cache_rows;
   a.rows = T * (H + 1);
   a.q_out = static_cast<uint8_t*>(q_out);

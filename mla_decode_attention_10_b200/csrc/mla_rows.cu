@@ -34,7 +34,7 @@ namespace rows {
 // Lanes per row and resident 256-thread blocks per SM the kernel is compiled
 // for.  e4m3 outputs: 16 lanes per row at 4 blocks (64 registers; measured on
 // B200 at T=8192, H=16: 40.1 us against 42.5 for one warp per row at 6
-// blocks and 41.0 at 5).  bf16 outputs: one warp per row at 5 blocks (48
+// blocks and 41.0 at 5).  bf16 outputs: one warp per row at 5 blocks (44
 // registers; 49.9 us at T=1024, H=128 against 53.4 for 16 lanes per row).
 __host__ __device__ constexpr int rows_lanes_per_row(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 16 : 32; }
 constexpr int rows_blocks_per_sm(bool qf8, bool kvf8) { return (qf8 || kvf8) ? 4 : 5; }
@@ -42,29 +42,14 @@ static_assert(rows_blocks_per_sm(true, true) <= kRowsMaxBlocksPerSm, "tuning lim
 
 // q / H for the row loop.  64-bit rows: one multiply-high by ceil(2^64 / H)
 // (div_heads).  32-bit rows (every call: T * (H + 1) < 2^31): with
-// 2^(s-1) < H <= 2^s and M = ceil(2^(31+s) / H) < 2^32,
-// floor(q M / 2^(31+s)) = floor(q / H) for 0 <= q < 2^31 (Granlund and
-// Montgomery, "Division by invariant integers using multiplication", PLDI
-// 1994), one 32-bit multiply-high and a shift.
-struct HeadDiv32 {
-  uint32_t m, shift;
-  bool one;
-};
-
-__device__ __forceinline__ HeadDiv32 head_div32(int64_t H) {
-  HeadDiv32 d;
-  d.one = H == 1;
-  const uint32_t s = d.one ? 1u : 32u - static_cast<uint32_t>(__clz(static_cast<int32_t>(H) - 1));
-  d.m = d.one ? 0u : static_cast<uint32_t>(((1ull << (31 + s)) + static_cast<uint64_t>(H) - 1) /
-                                           static_cast<uint64_t>(H));
-  d.shift = s - 1;
-  return d;
+// 2^(s-1) < H <= 2^s and M = ceil(2^(31+s) / H) < 2^32 (h_magic32, set by
+// the host), floor(q M / 2^(31+s)) = floor(q / H) for 0 <= q < 2^31
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994): one 32-bit multiply-high and a shift.
+__device__ __forceinline__ uint32_t div_h(const Args& a, uint32_t q) {
+  return a.h_magic32 == 0u ? q : __umulhi(q, a.h_magic32) >> a.h_shift32;
 }
-
-__device__ __forceinline__ uint32_t div_h(const HeadDiv32& d, const Args&, uint32_t q) {
-  return d.one ? q : __umulhi(q, d.m) >> d.shift;
-}
-__device__ __forceinline__ int64_t div_h(const HeadDiv32&, const Args& a, int64_t q) { return div_heads(a, q); }
+__device__ __forceinline__ int64_t div_h(const Args& a, int64_t q) { return div_heads(a, q); }
 
 // Idx: the integer type of the row loop.  e4m3 outputs use 32 bits, unsigned
 // so that the trip counter times rows per trip cannot wrap (rows < 2^31):
@@ -76,7 +61,6 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
   constexpr int kRowsPerTrip = 32 / L, kChunks = 64 / L, kPairs = 32 / L;
   const int ll = threadIdx.x & (L - 1);
   const Idx sub = static_cast<Idx>((threadIdx.x & 31) / L);
-  const HeadDiv32 hd = head_div32(a.H);
   const Idx H = static_cast<Idx>(a.H);
   const Idx T = static_cast<Idx>(a.T);
   const Idx rows = static_cast<Idx>(a.rows);
@@ -106,7 +90,7 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
       }
     } else {
       const Idx q = g - T;
-      t = div_h(hd, a, q);
+      t = div_h(a, q);
       const Idx h = q - t * H;
       nope = a.q_nope + static_cast<int64_t>(t) * a.qn_st + static_cast<int64_t>(h) * a.qn_sh;
       pe = a.q_pe + static_cast<int64_t>(t) * a.qp_st + static_cast<int64_t>(h) * a.qp_sh;
