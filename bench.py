@@ -66,11 +66,11 @@ KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
                   "mla_decode_attention_10_b200/csrc/mla_rows.cu",
                   "mla_decode_attention_10_b200/csrc/epilogue_device.cuh",
                   "mla_decode_attention_10_b200/csrc/latent_math.cuh", "include/mla_epilogue.h")
-TRAFFIC_SOURCE_HASH = "344ebd9364cf6c2b"
+TRAFFIC_SOURCE_HASH = "8201c5ad1fd365ce"
 TRAFFIC_BYTES = {
-    "batch_t8192_h16_pdl_fp8": 163928832 + 50717952,
+    "batch_t8192_h16_pdl_fp8": 163943680 + 51074560,
     "split_boundary_t64_h16_rope": 1279488 + 0,
-    "prefill_t1024_h128_strided": 152629760 + 101840128,
+    "prefill_t1024_h128_strided": 152632320 + 101192448,
 }
 L2_BYTES = 126 * 2 ** 20
 # The weight-streaming producer (decode sizes): the weights a projection

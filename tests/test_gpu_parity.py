@@ -252,6 +252,16 @@ def test_one_token_one_head_and_max_heads(force):
         check_workload(w, extra_flags=force)
 
 
+@pytest.mark.parametrize("force", FORCE[1:])
+@pytest.mark.parametrize("T,H", [(2, 65536), (3, 40009)])
+def test_largest_head_counts(force, T, H):
+    """The head count limit and a large odd one: (token, head) come from the
+    row index by a multiply-high division, exact over every row of a call."""
+    w = W.make("many_heads", T, H, W.FLAG_ROPE | W.FLAG_Q_FP8, seed=T + H, num_blocks=1, block_size=8,
+               rope_rows=64, scale=0.05, cache_fill="random")
+    check_workload(w, extra_flags=force)
+
+
 def test_misaligned_arguments_launch_nothing():
     w = W.make("align", 4, 4, 0, seed=2, num_blocks=1, cache_fill="random")
     d = w.to("cuda")
