@@ -41,6 +41,7 @@ struct Args {
   uint64_t h_magic;   // ceil(2^64 / H) for H >= 2, see div_heads
   uint32_t h_magic32;  // ceil(2^(31+s) / H), 2^(s-1) < H <= 2^s, for H >= 2; 0 for H = 1
   uint32_t h_shift32;  // s - 1
+  int32_t pe_vec;      // q_pe / k_pe rows 4-byte aligned and the table 8-byte aligned: pe pairs two at a time
   int64_t cache_rows;
   int64_t rows;  // T * (H + 1)
   uint8_t* q_out;
@@ -129,6 +130,39 @@ __device__ __forceinline__ void store_pe(uint8_t* dst, int i, uint32_t pe, const
     uint16_t* o = reinterpret_cast<uint16_t*>(dst);
     o[kNope + i] = static_cast<uint16_t>(p & 0xffffu);
     o[kNope + kHalfPe + i] = static_cast<uint16_t>(p >> 16);
+  }
+}
+
+// RoPE pairs i0 and i0 + 1 of a row together (i0 even): a01 holds pe[i0],
+// pe[i0+1] and b01 holds pe[i0+32], pe[i0+33]; the outputs go out as one
+// 2-byte (e4m3) or 4-byte (bf16) store per half.  r0 and r1 rotate pairs i0
+// and i0 + 1 (both on or both off: one position per token).
+template <bool FP8, bool ROPE, bool FAST>
+__device__ __forceinline__ void store_pe2(uint8_t* dst, int i0, uint32_t a01, uint32_t b01, const Rot& r0,
+                                          const Rot& r1, const Divisor& d) {
+  bool rotated = false;
+  float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
+  if constexpr (ROPE) {
+    if (r0.on) {
+      rope_pair(bf16_lo(a01), bf16_lo(b01), r0.c, r0.s, a0, b0);
+      rope_pair(bf16_hi(a01), bf16_hi(b01), r1.c, r1.s, a1, b1);
+      rotated = true;
+    }
+  }
+  if constexpr (FP8) {
+    uint32_t ea, eb;
+    if (rotated) {
+      ea = e4m3x2_of_f32<FAST>(a0, a1, d);
+      eb = e4m3x2_of_f32<FAST>(b0, b1, d);
+    } else {  // unrotated values are bf16: the quotient of bf16 inputs
+      ea = e4m3x2_of_bf16x2<FAST>(a01, d);
+      eb = e4m3x2_of_bf16x2<FAST>(b01, d);
+    }
+    *reinterpret_cast<uint16_t*>(dst + kNope + i0) = static_cast<uint16_t>(ea);
+    *reinterpret_cast<uint16_t*>(dst + kNope + kHalfPe + i0) = static_cast<uint16_t>(eb);
+  } else {
+    *reinterpret_cast<uint32_t*>(dst + 2 * (kNope + i0)) = rotated ? pack_bf16x2(a0, a1) : a01;
+    *reinterpret_cast<uint32_t*>(dst + 2 * (kNope + kHalfPe + i0)) = rotated ? pack_bf16x2(b0, b1) : b01;
   }
 }
 

@@ -341,6 +341,8 @@ mla_status mla_epilogue_launch(
   a.positions = positions;
   a.cos_sin = cos_sin;
   a.rope_rows = rope ? rope_rows : 0;
+  a.pe_vec = aligned(q_pe, 4) && aligned(k_pe, 4) && (T == 1 || (q_pe_stride_t % 2 == 0 && k_pe_stride_t % 2 == 0)) &&
+             (H == 1 || q_pe_stride_h % 2 == 0) && (!rope || aligned(cos_sin, 8));
   a.q_scale = q_scale;
   a.kv_scale = kv_scale;
   a.T = T;

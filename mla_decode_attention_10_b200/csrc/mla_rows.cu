@@ -56,8 +56,13 @@ __device__ __forceinline__ int64_t div_h(const Args& a, int64_t q) { return div_
 // the e4m3 kernel is bound by instruction issue, and 32-bit indexing saves a
 // tenth of its instructions (measured on B200: 47.2 -> 44.2 us at T=8192,
 // H=16); bf16 outputs, bound by memory, keep 64 bits (2% faster there).
-template <int L, typename Idx, bool QF8, bool KVF8, bool ROPE, bool FAST>
+// VEC (16 lanes per row, pe rows and table aligned): lane l takes the RoPE
+// pairs 2l and 2l + 1 with one 4-byte load per pe half, one 8-byte load each
+// of cos and sin, and one 2- or 4-byte store per pe half (store_pe2);
+// otherwise lane l takes pairs l + k L, one 2-byte load and one store each.
+template <int L, bool VEC, typename Idx, bool QF8, bool KVF8, bool ROPE, bool FAST>
 __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, const Divisor& dk) {
+  static_assert(!VEC || L == 16, "two pairs per lane cover a row at 16 lanes");
   constexpr int kRowsPerTrip = 32 / L, kChunks = 64 / L, kPairs = 32 / L;
   const int ll = threadIdx.x & (L - 1);
   const Idx sub = static_cast<Idx>((threadIdx.x & 31) / L);
@@ -103,11 +108,18 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
       const int32_t pos = __ldg(a.positions + t);
       if (pos >= 0 && pos < rope_rows) {
         const float* row = a.cos_sin + static_cast<int64_t>(pos) * kPe;
+        if constexpr (VEC) {
+          const float2 c = __ldg(reinterpret_cast<const float2*>(row) + ll);
+          const float2 sn = __ldg(reinterpret_cast<const float2*>(row + kHalfPe) + ll);
+          rot[0] = Rot{c.x, sn.x, true};
+          rot[1] = Rot{c.y, sn.y, true};
+        } else {
 #pragma unroll
-        for (int k = 0; k < kPairs; ++k) {
-          rot[k].c = __ldg(row + ll + k * L);
-          rot[k].s = __ldg(row + kHalfPe + ll + k * L);
-          rot[k].on = true;
+          for (int k = 0; k < kPairs; ++k) {
+            rot[k].c = __ldg(row + ll + k * L);
+            rot[k].s = __ldg(row + kHalfPe + ll + k * L);
+            rot[k].on = true;
+          }
         }
       }
       if (is_cache && ll == 0 && !rot[0].on) report(a.status, MLA_STATUS_POS_RANGE);
@@ -121,22 +133,35 @@ __device__ __forceinline__ void rows_body(const Args& a, const Divisor& dq, cons
 
     // 3. the row's loads, then 4. convert and store
     uint4 n[kChunks];
-    uint32_t p[kPairs];
+    uint32_t p[kPairs];  // VEC: p[0] = pe[2l], pe[2l+1]; p[1] = pe[2l+32], pe[2l+33]
 #pragma unroll
     for (int k = 0; k < kChunks; ++k) n[k] = ld_chunk(nope, ll + k * L);
+    if constexpr (VEC) {
+      p[0] = __ldcg(reinterpret_cast<const uint32_t*>(pe) + ll);
+      p[1] = __ldcg(reinterpret_cast<const uint32_t*>(pe + kHalfPe) + ll);
+    } else {
 #pragma unroll
-    for (int k = 0; k < kPairs; ++k) p[k] = ld_pair(pe, ll + k * L);
+      for (int k = 0; k < kPairs; ++k) p[k] = ld_pair(pe, ll + k * L);
+    }
     if (dst == nullptr) continue;
     if (is_cache) {
 #pragma unroll
       for (int k = 0; k < kChunks; ++k) store_nope<KVF8, FAST>(dst, ll + k * L, n[k], dk);
+      if constexpr (VEC) {
+        store_pe2<KVF8, ROPE, FAST>(dst, 2 * ll, p[0], p[1], rot[0], rot[1], dk);
+      } else {
 #pragma unroll
-      for (int k = 0; k < kPairs; ++k) store_pe<KVF8, ROPE, FAST>(dst, ll + k * L, p[k], rot[k], dk);
+        for (int k = 0; k < kPairs; ++k) store_pe<KVF8, ROPE, FAST>(dst, ll + k * L, p[k], rot[k], dk);
+      }
     } else {
 #pragma unroll
       for (int k = 0; k < kChunks; ++k) store_nope<QF8, FAST>(dst, ll + k * L, n[k], dq);
+      if constexpr (VEC) {
+        store_pe2<QF8, ROPE, FAST>(dst, 2 * ll, p[0], p[1], rot[0], rot[1], dq);
+      } else {
 #pragma unroll
-      for (int k = 0; k < kPairs; ++k) store_pe<QF8, ROPE, FAST>(dst, ll + k * L, p[k], rot[k], dq);
+        for (int k = 0; k < kPairs; ++k) store_pe<QF8, ROPE, FAST>(dst, ll + k * L, p[k], rot[k], dq);
+      }
     }
   }
 }
@@ -151,10 +176,15 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps, rows_blocks_per_sm(QF8, KV
   if constexpr (KVF8) dk = make_divisor(__ldg(a.kv_scale));
   using Idx = std::conditional_t<QF8 || KVF8, uint32_t, int64_t>;
   constexpr int L = rows_lanes_per_row(QF8, KVF8);
+  constexpr bool kCanVec = L == 16;
   if (dq.fast && dk.fast) {
-    rows_body<L, Idx, QF8, KVF8, ROPE, true>(a, dq, dk);
+    if (kCanVec && a.pe_vec) {
+      rows_body<L, kCanVec, Idx, QF8, KVF8, ROPE, true>(a, dq, dk);
+    } else {
+      rows_body<L, false, Idx, QF8, KVF8, ROPE, true>(a, dq, dk);
+    }
   } else {
-    rows_body<L, Idx, QF8, KVF8, ROPE, false>(a, dq, dk);
+    rows_body<L, false, Idx, QF8, KVF8, ROPE, false>(a, dq, dk);
   }
   pdl_trigger();
 }

@@ -90,12 +90,17 @@ def _shift_view(t: torch.Tensor, elems: int) -> torch.Tensor:
 
 @pytest.mark.parametrize("force", FORCE)
 @pytest.mark.parametrize("T", [1, 9, 300])
-def test_unaligned_pe_rows_and_table(force, T):
+@pytest.mark.parametrize("pe_shift,k_shift,table_shift", [(1, 3, 1), (2, 2, 1), (2, 6, 2)])
+def test_unaligned_pe_rows_and_table(force, T, pe_shift, k_shift, table_shift):
+    """q_pe / k_pe rows and the cos/sin table off the 16-byte grid: 2-byte
+    aligned pe (one element pairs at a time), 4-byte aligned pe with a 4-byte
+    aligned table (still one pair at a time), and 4-byte pe with an 8-byte
+    aligned table (the rows kernel takes two pairs per lane)."""
     w = W.make("unaligned", T, 16, W.FLAG_ROPE | W.FLAG_Q_FP8, seed=70 + T, num_blocks=8, std=2.0, rope_rows=512,
                scale=0.05, cache_fill="random")
-    w.q_pe = _shift_view(w.q_pe.contiguous(), 1)     # 2-byte aligned rows
-    w.k_pe = _shift_view(w.k_pe.contiguous(), 3)
-    w.cos_sin = _shift_view(w.cos_sin, 1)            # 4-byte aligned table rows
+    w.q_pe = _shift_view(w.q_pe.contiguous(), pe_shift)
+    w.k_pe = _shift_view(w.k_pe.contiguous(), k_shift)
+    w.cos_sin = _shift_view(w.cos_sin, table_shift)
     assert w.q_pe.data_ptr() % 16 and w.k_pe.data_ptr() % 16 and w.cos_sin.data_ptr() % 16
     check_workload(w, extra_flags=force)
 
@@ -104,8 +109,7 @@ def test_unaligned_pe_rows_and_table(force, T):
 
 @pytest.mark.parametrize("warps", [1, 3, 8])
 def test_rows_kernel_warp_counts(warps):
-    """Blocks of 1 .. 8 warps; every warp walks many rows, so its four-slot
-    ring wraps many times."""
+    """Blocks of 1 .. 8 warps; every warp walks many rows."""
     old = E.mla_epilogue_get_tuning()
     try:
         E.mla_epilogue_set_tuning(rows_warps_per_block=warps)
