@@ -7,7 +7,9 @@
 // adjacent rows per trip (L lanes each) and then moves on by the number of
 // warps in the grid, so all warps walk one window of memory together.  Lane l
 // of a row moves nope chunks l + k L (16 bytes each) and rotates the pe pairs
-// (i, i + 32) for i = l + k L.  With an e4m3 output L = 16: the kernel is
+// (i, i + 32) for i = l + k L, or, with L = 16 and the pe rows and the table
+// aligned, for i = 2l and 2l + 1 (vector loads and stores; the launcher sets
+// pe_vec).  With an e4m3 output L = 16: the kernel is
 // bound by instruction issue (measured on B200), and two rows per warp trip
 // halve the per-row instructions (addresses, slot, position, table row,
 // checks) while the e4m3 arithmetic stays spread over all 32 lanes.  bf16
