@@ -66,11 +66,11 @@ KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
                   "mla_decode_attention_10_b200/csrc/mla_rows.cu",
                   "mla_decode_attention_10_b200/csrc/epilogue_device.cuh",
                   "mla_decode_attention_10_b200/csrc/latent_math.cuh", "include/mla_epilogue.h")
-TRAFFIC_SOURCE_HASH = "8201c5ad1fd365ce"
+TRAFFIC_SOURCE_HASH = "ad10677baa8ce97d"
 TRAFFIC_BYTES = {
-    "batch_t8192_h16_pdl_fp8": 163943680 + 51074560,
-    "split_boundary_t64_h16_rope": 1279488 + 0,
-    "prefill_t1024_h128_strided": 152632320 + 101192448,
+    "batch_t8192_h16_pdl_fp8": 163964672 + 49944320,
+    "split_boundary_t64_h16_rope": 1279232 + 0,
+    "prefill_t1024_h128_strided": 152633344 + 101662464,
 }
 L2_BYTES = 126 * 2 ** 20
 # The weight-streaming producer (decode sizes): the weights a projection
@@ -349,6 +349,17 @@ def flush_l2():
 # our implementation
 # ---------------------------------------------------------------------------------------
 
+def interleaved_medians(runners: dict, device, calls: int, reps: int) -> dict:
+    """Median µs per call of each runner over `reps` timed regions, the runners
+    taking turns within every repetition, so that a drift of the clocks
+    between repetitions lands on all of them alike."""
+    times = {k: [] for k in runners}
+    for _ in range(reps):
+        for k, r in runners.items():
+            times[k].append(job_us_per_call(timed(r, device), calls, 1))
+    return {k: statistics.median(v) for k, v in times.items()}
+
+
 def median_us(runner, device, calls: int, reps: int, world: int = 1, flush: bool = True) -> float:
     """Median over `reps` timed regions of one replay each, as whole-job
     microseconds per call (each region's time is the max over ranks)."""
@@ -457,11 +468,9 @@ def behind_producer(hx, ds, device, calls, reps, prod=None, prefix=""):
              "producer_epilogue_no_pdl_us": then(prod, hx.epilogue(ds)),
              "producer_empty_pdl_us": then(prod, empty),
              "producer_empty_wait_pdl_us": then(prod, empty_wait)}
-    out = {}
-    for key, fn in steps.items():
-        r = hx.runner(fn, calls)
-        out[key] = round(median_us(r, device, calls, reps), 4)
-        del r
+    runners = {key: hx.runner(fn, calls) for key, fn in steps.items()}
+    out = {k: round(v, 4) for k, v in interleaved_medians(runners, device, calls, reps).items()}
+    del runners
     p = out["producer_us"]
     inc = out["producer_epilogue_pdl_us"] - p
     inc_wait = out["producer_empty_wait_pdl_us"] - p
@@ -480,13 +489,10 @@ def standalone(hx, ds, device, calls, reps, peak):
     w0 = ds.w0
     if calls is None:
         calls = 20 if ds.bytes_per_call > 32 * 2 ** 20 else 200
-    r = hx.runner(hx.epilogue(ds), calls)
-    us = median_us(r, device, calls, reps)
-    del r
     fstep, plan = hx.empty(w0, 0)
-    fr = hx.runner(fstep, calls)
-    floor_us = median_us(fr, device, calls, reps)
-    del fr
+    m = interleaved_medians({"epilogue": hx.runner(hx.epilogue(ds), calls), "empty": hx.runner(fstep, calls)},
+                            device, calls, reps)
+    us, floor_us = m["epilogue"], m["empty"]
     gbs = w0.algorithmic_bytes() / (us * 1e-6) / 1e9
     return {"workload": ds.name, "T": w0.T, "H": w0.H, "flags": flag_names(w0.flags), "mode": mode_name(hx.E, plan),
             "grid": [plan.blocks, plan.threads_per_block], "bytes_per_call": w0.algorithmic_bytes(),
