@@ -119,7 +119,9 @@ typedef enum mla_status {
  * (2-byte) alignment; slot_mapping 8 bytes; positions, cos_sin, scales and
  * status 4 bytes.  Strides must be >= 0.  Otherwise MLA_ERR_ALIGNMENT or
  * MLA_ERR_INVALID_ARG and nothing is launched.  Sizes: H <= 65536 and
- * T * (H + 1) < 2^31.
+ * T * (H + 1) < 2^31.  With q_pe and k_pe rows 4-byte aligned (even strides)
+ * and cos_sin 8-byte aligned, MLA_MODE_ROWS with an e4m3 output reads and
+ * writes the pe values as vectors; the results are the same either way.
  *
  * Programmatic dependent launch (MLA_FLAG_PDL, as the enable_pdl argument of
  * the vLLM PR #54565 report's GEMM entry): the kernel may start before the
