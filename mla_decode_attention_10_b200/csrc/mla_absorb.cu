@@ -1,9 +1,15 @@
 // mla_absorb.cu -- latent query rows straight from the absorption product, on
 // the tcgen05 tensor cores (contract in mla_absorb.h).
 //
-// A persistent kernel, one CTA per SM, that takes a contiguous run of
-// 128-token x 256-column tiles in (head, column half, token tile) order, so a
-// head's weights are loaded once for many token tiles.  Its warps have roles:
+// A persistent kernel, one CTA per SM, over 128-token x 256-column tiles.
+// When the 2H (head, column half) pairs fit the grid, each pair gets
+// grid / 2H CTAs that take every (grid / 2H)-th token tile of it, and the
+// grid % 2H remaining CTAs share out the last token tiles of every pair: a
+// CTA loads its weights once, and the running CTAs read all heads of the
+// same token tiles together, which keeps DRAM pages open (measured on B200
+// at T=8192, H=16, e4m3: 36.6 -> 34.9 us).  Otherwise each CTA takes a
+// contiguous run of tiles in (head, column half, token tile) order.  Its
+// warps have roles:
 //   * warp 0 (TMA): per tile, the A tile (q_nope_c: 128 tokens x 128) into a
 //     two-stage ring and, when the (head, column half) changes, the B tile
 //     (w_uk: 256 latent rows x 128), both with the 128-byte swizzle; the
@@ -79,6 +85,9 @@ struct Params {
   int32_t* status;
   int32_t pe_vec;   // q_pe rows may be read as 16-byte vectors
   int32_t tab_vec;  // cos_sin rows may be read as 16-byte vectors
+  int32_t strided;    // 2H <= grid: the per-(head, half) assignment above, else contiguous runs
+  int32_t per_combo;  // main CTAs per (head, half): CTA c < per_combo * 2H takes pair c mod 2H
+  int32_t tail;       // last token tiles of every pair, shared out to the CTAs past the main ones
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -326,7 +335,7 @@ __device__ __forceinline__ bool bar_and(int id, int n, bool pred) {
 
 __device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-// Tile order: (head, column half, token tile), token tile fastest.
+// Contiguous-run tile order: (head, column half, token tile), token tile fastest.
 struct TileCoord {
   int h, nt, m0;
 };
@@ -358,8 +367,30 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
   const int per = tiles / static_cast<int>(gridDim.x);
   const int rem = tiles - per * static_cast<int>(gridDim.x);
   const int bx = static_cast<int>(blockIdx.x);
-  const int first = bx * per + (bx < rem ? bx : rem);
-  const int count = per + (bx < rem ? 1 : 0);
+  const int combos = 2 * p.H;
+  const int mains = p.per_combo * combos;
+  const int mm = mt - p.tail;  // token tiles of the main part
+  const bool main_cta = p.strided && bx < mains;
+  const bool extra_cta = p.strided && bx >= mains;
+  const int combo = bx % combos, j0 = bx / combos, step = p.per_combo;
+  const int extras = static_cast<int>(gridDim.x) - mains;
+  const int tail_tiles = p.tail * combos;
+  const int e = bx - mains;
+  const int lo = extra_cta ? static_cast<int>(static_cast<int64_t>(e) * tail_tiles / extras) : 0;
+  const int hi = extra_cta ? static_cast<int>(static_cast<int64_t>(e + 1) * tail_tiles / extras) : 0;
+  const int first = p.strided ? 0 : bx * per + (bx < rem ? bx : rem);
+  const int count = main_cta ? (j0 < mm ? (mm - j0 + step - 1) / step : 0)
+                    : extra_cta ? hi - lo
+                                : per + (bx < rem ? 1 : 0);
+  auto coord = [&](int i) -> TileCoord {
+    if (main_cta) return TileCoord{combo >> 1, combo & 1, (j0 + i * step) * kM};
+    if (extra_cta) {
+      const int tau = lo + i;  // tail tiles in (head, half)-major order
+      const int cb = tau / p.tail;
+      return TileCoord{cb >> 1, cb & 1, (mm + tau - cb * p.tail) * kM};
+    }
+    return tile_at(first + i, mt);
+  };
   const uint32_t sB = sbase;
   const uint32_t sA = sbase + kBBytes;
   const uint32_t sC = sA + kStages * kABytes;
@@ -369,7 +400,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
       bool waited = false;
       int group = -1, groups = 0, issued = 0;
       for (int i = 0; i < count && *abort_flag == 0u; ++i) {
-        const TileCoord c = tile_at(first + i, mt);
+        const TileCoord c = coord(i);
         const int g = c.h * 2 + c.nt;
         if (g != group) {
           if (groups > 0 && !wait_or_abort(smem_u32(&bars.b_empty), static_cast<uint32_t>(groups - 1) & 1u, abort_flag)) {
@@ -411,7 +442,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
     if (lane == 0) {
       int group = -1, groups = 0;
       for (int i = 0; i < count && *abort_flag == 0u; ++i) {
-        const TileCoord c = tile_at(first + i, mt);
+        const TileCoord c = coord(i);
         const int g = c.h * 2 + c.nt;
         if (g != group) {
           if (!wait_or_abort(smem_u32(&bars.b_full), static_cast<uint32_t>(groups) & 1u, abort_flag)) {
@@ -447,7 +478,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
                      : "memory");
         bool last_of_group = (i + 1 == count);
         if (!last_of_group) {
-          const TileCoord n = tile_at(first + i + 1, mt);
+          const TileCoord n = coord(i + 1);
           last_of_group = (n.h * 2 + n.nt) != g;
         }
         if (last_of_group)
@@ -469,7 +500,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmA, const CUtensorMap* t
     const bool issuer = (ew & 3) == 0 && lane == 0;  // issues the bulk stores of its half
     constexpr int kSlabCols = QF8 ? 128 : 64;
     for (int i = 0; i < count; ++i) {
-      const TileCoord c = tile_at(first + i, mt);
+      const TileCoord c = coord(i);
       const int b = i & 1;
       // lane 0 polls for its warp; the barrier below orders the other lanes
       // after its wait, and the tcgen05 fence after the barrier orders the
@@ -707,6 +738,21 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
   prm.status = status;
   prm.pe_vec = aligned(q_pe, 16) && (T == 1 || qp_st % 8 == 0) && (H == 1 || qp_sh % 8 == 0);
   prm.tab_vec = rope && aligned(cos_sin, 16);
+  prm.strided = (2 * H <= sms) ? 1 : 0;
+  prm.per_combo = prm.strided ? static_cast<int32_t>(sms / (2 * H)) : 1;
+  prm.tail = 0;
+  if (prm.strided) {
+    // tail tiles per (head, half) that balance the main CTAs against the extras
+    const int64_t mt = (T + kM - 1) / kM, C = 2 * H, E = sms - prm.per_combo * C;
+    int64_t best = -1, best_span = INT64_MAX;
+    for (int64_t tl = 0; tl <= (E > 0 ? mt : 0); ++tl) {
+      const int64_t main_span = (mt - tl + prm.per_combo - 1) / prm.per_combo;
+      const int64_t extra_span = E > 0 ? (tl * C + E - 1) / E : 0;
+      const int64_t span = main_span > extra_span ? main_span : extra_span;
+      if (span < best_span) { best_span = span; best = tl; }
+    }
+    prm.tail = static_cast<int32_t>(best);
+  }
 
   const int k = (qf8 ? 2 : 0) | (rope ? 1 : 0);
   static const void* const kernels[4] = {kernel_for<false, false>(), kernel_for<false, true>(),
@@ -722,7 +768,9 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
 
   cudaLaunchConfig_t cfg = {};
   const int64_t tiles = 2 * H * ((T + kM - 1) / kM);
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms), 1, 1);
+  int64_t grid = tiles < sms ? tiles : sms;
+  if (prm.strided) grid = prm.tail > 0 ? sms : prm.per_combo * 2 * H;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
