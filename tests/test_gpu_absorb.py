@@ -85,6 +85,18 @@ def test_absorbed_rows_named_workloads():
         _check(w, q, st)
 
 
+@pytest.mark.parametrize("flags", [W.FLAG_ROPE, W.FLAG_ROPE | W.FLAG_Q_FP8])
+@pytest.mark.parametrize("T,H", [(600, 40), (200, 80)])
+def test_absorbed_rows_tile_assignments(flags, T, H):
+    """(600, 40): one CTA per (head, half) takes the first token tiles, the
+    other CTAs share out the last two of every pair, several pairs each (so
+    their weights change between tiles).  (200, 80): more (head, half) pairs
+    than SMs, so CTAs take contiguous runs of tiles."""
+    w = W.make_absorb("assign", T, H, flags, seed=T + H + flags, rope_rows=4096, scale=0.05)
+    q, st = _gpu(w)
+    _check(w, q, st)
+
+
 def test_identity_weights_copy_bit_for_bit():
     w = W.make_absorb("id", 200, 4, W.FLAG_ROPE, seed=5, rope_rows=512)
     w.w_uk.zero_()
