@@ -742,14 +742,21 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
   prm.per_combo = prm.strided ? static_cast<int32_t>(sms / (2 * H)) : 1;
   prm.tail = 0;
   if (prm.strided) {
-    // tail tiles per (head, half) that balance the main CTAs against the extras
-    const int64_t mt = (T + kM - 1) / kM, C = 2 * H, E = sms - prm.per_combo * C;
-    int64_t best = -1, best_span = INT64_MAX;
-    for (int64_t tl = 0; tl <= (E > 0 ? mt : 0); ++tl) {
-      const int64_t main_span = (mt - tl + prm.per_combo - 1) / prm.per_combo;
-      const int64_t extra_span = E > 0 ? (tl * C + E - 1) / E : 0;
-      const int64_t span = main_span > extra_span ? main_span : extra_span;
-      if (span < best_span) { best_span = span; best = tl; }
+    // tail tiles per (head, half) that balance the main CTAs, (mt - tail) / R
+    // tiles each, against the E extras, tail * 2H / E each: the balance point
+    // mt E / (E + R 2H), and its neighbours for the rounding
+    const int64_t mt = (T + kM - 1) / kM, C = 2 * H, R = prm.per_combo, E = sms - R * C;
+    int64_t best = 0, best_span = (mt + R - 1) / R;
+    if (E > 0) {
+      const int64_t t0 = mt * E / (E + R * C);
+      for (int64_t tl = t0 > 2 ? t0 - 2 : 0; tl <= t0 + 3 && tl <= mt; ++tl) {
+        const int64_t main_span = (mt - tl + R - 1) / R, extra_span = (tl * C + E - 1) / E;
+        const int64_t span = main_span > extra_span ? main_span : extra_span;
+        if (span < best_span) {
+          best_span = span;
+          best = tl;
+        }
+      }
     }
     prm.tail = static_cast<int32_t>(best);
   }
