@@ -514,7 +514,8 @@ def decode_floors(hx, device, peak, calls=200, reps=7):
     as the projection that produces q would.  `floor_ratio_behind_producer`
     is the epilogue's increment over the producer against the increment of
     an empty dependent that waits, `increment_over_launch_floor` the same
-    increment against one bare launch of an empty kernel."""
+    increment against one bare launch of an empty kernel (the median over the
+    sizes, `launch_floor_median_us`)."""
     out = []
     pool = torch.ones(GEMM_WEIGHT_POOL_BYTES // 4, dtype=torch.int32, device=device)
     sink = torch.zeros(1, dtype=torch.int32, device=device)
@@ -523,14 +524,19 @@ def decode_floors(hx, device, peak, calls=200, reps=7):
         row = standalone(hx, ds, device, calls, reps, peak)
         row.update(behind_producer(hx, ds, device, calls, reps))
         row.update(behind_producer(hx, ds, device, calls, reps, hx.producer_after_weights(ds, pool, sink), "gemm_"))
-        # the epilogue's cost behind each producer against one bare launch
-        row["increment_over_launch_floor"] = round(row["epilogue_increment_pdl_us"] / row["launch_floor_us"], 3)
-        row["gemm_increment_over_launch_floor"] = round(row["gemm_epilogue_increment_pdl_us"] /
-                                                        row["launch_floor_us"], 3)
         out.append(row)
         del ds
         torch.cuda.empty_cache()
     del pool, sink
+    # the epilogue's cost behind each producer against one bare launch: the
+    # median over these sizes of the empty kernel's time (the grids differ
+    # little; a replay of the empty kernel now and then runs a third faster,
+    # and one such reading should not decide a ratio it was not timed with)
+    floor = statistics.median(r["launch_floor_us"] for r in out)
+    for r in out:
+        r["launch_floor_median_us"] = round(floor, 4)
+        r["increment_over_launch_floor"] = round(r["epilogue_increment_pdl_us"] / floor, 3)
+        r["gemm_increment_over_launch_floor"] = round(r["gemm_epilogue_increment_pdl_us"] / floor, 3)
     return out
 
 
