@@ -66,7 +66,7 @@ KERNEL_SOURCES = ("mla_decode_attention_10_b200/csrc/mla_epilogue.cu",
                   "mla_decode_attention_10_b200/csrc/mla_rows.cu",
                   "mla_decode_attention_10_b200/csrc/epilogue_device.cuh",
                   "mla_decode_attention_10_b200/csrc/latent_math.cuh", "include/mla_epilogue.h")
-TRAFFIC_SOURCE_HASH = "e083ffdaf79dc620"
+TRAFFIC_SOURCE_HASH = "c179ba93f29fcdba"
 TRAFFIC_BYTES = {
     "batch_t8192_h16_pdl_fp8": 163964672 + 49944320,
     "split_boundary_t64_h16_rope": 1279232 + 0,

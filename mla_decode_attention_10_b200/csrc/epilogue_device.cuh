@@ -73,10 +73,11 @@ __device__ __forceinline__ Divisor divisor_of(const float* scale) {
   return d;
 }
 
-// ---- one row, a warp-wide slice at a time: lane l moves 16-byte nope chunk
-// c and rotates pe pair (l, l + 32).  Loads of data the upstream kernel may
-// still be writing under programmatic dependent launch go to L2 only (.cg),
-// never through the read-only path.
+// ---- pieces of one row: a 16-byte nope chunk (8 values) and the RoPE pairs
+// (i, i + 32), one pair (store_pe) or two adjacent pairs (store_pe2) at a
+// time; the kernels decide which lane takes which piece.  Loads of data the
+// upstream kernel may still be writing under programmatic dependent launch go
+// to L2 only (.cg), never through the read-only path.
 
 // Rotation of pair `i` for token t: (cos, sin) from the table row of its
 // position, or `on` false when the position is out of range.
@@ -173,10 +174,5 @@ __device__ __forceinline__ uint4 ld_chunk(const uint16_t* row, int chunk) {
 __device__ __forceinline__ uint32_t ld_pair(const uint16_t* pe, int i) {
   return static_cast<uint32_t>(__ldcg(pe + i)) | (static_cast<uint32_t>(__ldcg(pe + kHalfPe + i)) << 16);
 }
-
-// ------------------------------------------------------------------------------------
-// rows kernel: one warp per row, grid-stride over rows
-// ------------------------------------------------------------------------------------
-
 
 }  // namespace mla

@@ -1,5 +1,5 @@
 // mla_epilogue.cu -- the fused MLA decode epilogue for B200 (sm_100a): the
-// small-batch kernels and the C-ABI launcher.
+// small-batch kernel and the C-ABI launcher.
 //
 // Per token t: H latent query rows q_out[t, h] = enc(rope(q_nope[t, h] || q_pe[t, h]))
 // and one latent cache row cache[slot_mapping[t]] = enc(rope(kv_c[t] || k_pe[t])),
@@ -8,7 +8,7 @@
 //
 // The op moves bytes and does almost no arithmetic: at decode sizes it is
 // bound by launch and memory latency, at large T by HBM bandwidth; there is
-// no contraction and no tensor-core work.  Three launch modes:
+// no contraction and no tensor-core work.  Two launch modes:
 //
 //   SPLIT (small T): every row gets three warps, as the page's SPLIT=3 path
 //     does.  Warps 0 and 1 move the 64 nope chunks (16 bytes, 8 values, one
