@@ -4,10 +4,11 @@
  * conventions: device pointers owned by the caller, asynchronous on
  * `stream`, nothing allocated, host argument errors returned as mla_status).
  *
- * None of these is part of the epilogue itself; they exist to put it in the
- * setting the vLLM PR #54896 report describes (an upstream producer kernel
- * linked by programmatic dependent launch, 实现拆解 item 2), to time a bare
- * launch, and to check the e4m3 quotient on the device.
+ * None of these is part of the epilogue itself.  They put it in the setting
+ * the vLLM PR #54896 report describes: an upstream producer kernel, linked
+ * by programmatic dependent launch (实现拆解 item 2), and a downstream
+ * consumer.  They also time a bare launch, and check the e4m3 quotient on
+ * the device.
  */
 #ifndef MLA_HARNESS_H
 #define MLA_HARNESS_H

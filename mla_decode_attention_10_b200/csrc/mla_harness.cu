@@ -1,5 +1,7 @@
-// mla_harness.cu -- synthetic producer, bare-launch kernel and quotient self-check
-// that sit beside the epilogue (declarations and contracts in mla_harness.h).
+// mla_harness.cu -- the kernels that sit beside the epilogue: synthetic
+// producers (copy-only, or streaming a weight buffer first), empty kernels for
+// the launch floors, a synthetic consumer, and two device checks of the e4m3
+// quotient (declarations and contracts in mla_harness.h).
 
 #include <cstdint>
 #include <cuda_fp16.h>
