@@ -46,7 +46,7 @@ extern "C" {
  *   q_pe      bf16 [T, H, 64] at (q_pe_stride_t, q_pe_stride_h, 1), 2-byte aligned.
  *   positions, cos_sin, rope_rows, q_scale: as in mla_epilogue_launch
  *             (flags MLA_FLAG_ROPE, MLA_FLAG_Q_FP8).
- *   T >= 0, 1 <= H <= 65535.
+ *   T >= 0, 1 <= H <= 65535, T * H <= 2^31 - 1 - 128.
  *   q_out     [T, H, 576] contiguous, bf16 or e4m3 bytes, 16-byte aligned.
  *   status    optional device int32: MLA_STATUS_POS_RANGE, MLA_STATUS_TIMEOUT.
  *   flags     MLA_FLAG_ROPE, MLA_FLAG_Q_FP8, MLA_FLAG_PDL (the q inputs come

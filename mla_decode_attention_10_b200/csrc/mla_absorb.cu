@@ -660,7 +660,9 @@ mla_status mla_absorb_launch(const void* q_nope_c, int64_t qc_st, int64_t qc_sh,
                              void* q_out, int32_t* status, mla_stream_t stream) {
   using namespace mla::absorb;
   if ((flags & ~(MLA_FLAG_ROPE | MLA_FLAG_Q_FP8 | MLA_FLAG_PDL)) != 0) return MLA_ERR_UNSUPPORTED;
-  if (T < 0 || H < 1 || H > 65535 || T > static_cast<int64_t>(INT_MAX) / H) return MLA_ERR_INVALID_ARG;
+  // T * H < 2^31 - 128: every token, tile and row index of the kernel (T rounded up to a whole tile
+  // included) stays in 32 bits
+  if (T < 0 || H < 1 || H > 65535 || T > (static_cast<int64_t>(INT_MAX) - kM) / H) return MLA_ERR_INVALID_ARG;
   const bool rope = (flags & MLA_FLAG_ROPE) != 0;
   const bool qf8 = (flags & MLA_FLAG_Q_FP8) != 0;
   if (rope && (rope_rows < 1 || rope_rows > (INT64_C(1) << 40))) return MLA_ERR_INVALID_ARG;

@@ -237,6 +237,7 @@ def test_harness_validation(lib, kw, code):
     (dict(T=-1), E.MLA_ERR_INVALID_ARG),
     (dict(H=0), E.MLA_ERR_INVALID_ARG),
     (dict(H=65536), E.MLA_ERR_INVALID_ARG),
+    (dict(H=1, T=2 ** 31 - 100), E.MLA_ERR_INVALID_ARG),
     (dict(q_nope_c=None), E.MLA_ERR_INVALID_ARG),
     (dict(w_uk=None), E.MLA_ERR_INVALID_ARG),
     (dict(q_out=None), E.MLA_ERR_INVALID_ARG),
